@@ -1,0 +1,54 @@
+"""CPU oracle: one multi-stream decode step against an interleaved KV cache.
+
+TEST INFRASTRUCTURE ONLY; the library never calls it.
+
+Sources (page "微信WeLM提出Hidden Decoding：大模型推理新范式", tahou.com):
+  * section "实验效果与成本分析": the n streams of a new token are computed in one
+    parallel forward, not one after another;
+  * section "中间流的作用验证": each stream keeps its own KV state;
+  * the mask is the prefill mask of the same layer type (section
+    "规模化落地的工程优化").
+
+Reading (pages silent on the cache layout): the cache holds the expanded
+sequence in position order, [B, Tcap*n, Hkv, D]; seqlen[b] counts tokens
+including the new one, whose n rows are already written at positions
+T*n .. T*n+n-1 (T = seqlen[b]-1). Query (s, h) of sequence b sits at p = T*n+s
+and reads cache positions p' < seqlen[b]*n that the layer's mask allows.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from .attention import CROSS_WINDOW, _f64, visible
+
+
+def decode_attn(q, k_cache, v_cache, seqlen, n, mode, W, scale):
+    """q [B, n, Hq, D]; caches [B, Tcap*n, Hkv, D]; seqlen int [B].
+
+    Returns (o [B, n, Hq, D], lse [B, Hq, n]) in float64.
+    """
+    q = _f64(q)
+    seqlen = np.asarray(seqlen.cpu() if hasattr(seqlen, "cpu") else seqlen, dtype=np.int64)
+    B, nn, Hq, D = q.shape
+    assert nn == n
+    Hkv = k_cache.shape[2]
+    g = Hq // Hkv
+    o = np.zeros((B, n, Hq, D))
+    lse = np.zeros((B, Hq, n))
+    for b in range(B):
+        T = int(seqlen[b]) - 1
+        for s in range(n):
+            p = T * n + s
+            lo = max(0, p - n * W + 1) if mode == CROSS_WINDOW else 0
+            keys = np.arange(lo, p + 1)
+            keys = keys[visible(p, keys, n, mode, W)]
+            for kh in range(Hkv):
+                kk = _f64(k_cache[b, keys, kh, :])
+                vv = _f64(v_cache[b, keys, kh, :])
+                for h in range(kh * g, (kh + 1) * g):
+                    sc = scale * (kk @ q[b, s, h])
+                    mx = sc.max()
+                    e = np.exp(sc - mx)
+                    lse[b, h, s] = mx + np.log(e.sum())
+                    o[b, s, h] = (e / e.sum()) @ vv
+    return o, lse

@@ -120,37 +120,44 @@ def attn_fwd(q, k, v, n, mode, W, final_only, scale):
     return o, lse
 
 
-def attn_fwd_rows(q, k, v, n, mode, W, final_only, scale, b, h, rows):
-    """Forward for selected query rows of one (batch, query head).
+def _row_block(q, k, v, n, mode, W, final_only, scale, b, h, rows):
+    """Scores of selected query rows against the keys they can reach.
 
-    ``rows`` index the query dimension of q (0..Sq-1). Returns
-    (o [len(rows), D], lse [len(rows)]), both float64. Each row only touches the
-    keys it can see, so this is cheap at any sequence length.
+    Returns (Q rows, K, V, P, lse) in float64 for the key window
+    [lo, hi) that covers every selected row; P is the masked softmax.
     """
     S, Hkv = k.shape[1], k.shape[2]
     Hq = q.shape[2]
     kh = h // (Hq // Hkv)
-    qpos_all = query_positions(S, n, final_only)
     rows = np.asarray(rows, dtype=np.int64)
-    qr = _f64(q[b, rows, h, :])
-    D = qr.shape[-1]
+    qpos = query_positions(S, n, final_only)[rows]
+    lo = max(0, int(qpos.min()) - n * W + 1) if mode == CROSS_WINDOW else 0
+    hi = int(qpos.max()) + 1
+    keys = np.arange(lo, hi)
+    mask = visible(qpos[:, None], keys[None, :], n, mode, W)
+    Q = _f64(q[b, rows, h, :])
+    K = _f64(k[b, lo:hi, kh, :])
+    V = _f64(v[b, lo:hi, kh, :])
+    P, lse = _rows_softmax(scale * (Q @ K.T), mask)
+    return Q, K, V, P, lse, lo
+
+
+def attn_fwd_rows(q, k, v, n, mode, W, final_only, scale, b, h, rows, block=64):
+    """Forward for selected query rows of one (batch, query head).
+
+    ``rows`` index the query dimension of q (0..Sq-1). Returns
+    (o [len(rows), D], lse [len(rows)]), both float64. Rows are taken in blocks
+    so the score matrix stays small at any sequence length.
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    D = q.shape[-1]
     o = np.zeros((len(rows), D))
     lse = np.zeros(len(rows))
-    for i, r in enumerate(rows):
-        p = int(qpos_all[r])
-        lo = 0
-        if mode == CROSS_WINDOW:
-            lo = max(0, p - n * W + 1)
-        keys = np.arange(lo, p + 1)
-        keys = keys[visible(p, keys, n, mode, W)]
-        kk = _f64(k[b, keys, kh, :])
-        vv = _f64(v[b, keys, kh, :])
-        sc = scale * (kk @ qr[i])
-        mx = sc.max()
-        e = np.exp(sc - mx)
-        tot = e.sum()
-        lse[i] = mx + np.log(tot)
-        o[i] = (e / tot) @ vv
+    for i in range(0, len(rows), block):
+        sel = rows[i:i + block]
+        _, _, V, P, l, _ = _row_block(q, k, v, n, mode, W, final_only, scale, b, h, sel)
+        o[i:i + block] = P @ V
+        lse[i:i + block] = l
     return o, lse
 
 
@@ -185,35 +192,23 @@ def attn_bwd(q, k, v, do, n, mode, W, final_only, scale):
     return dq, dk, dv
 
 
-def attn_bwd_dq_rows(q, k, v, do, n, mode, W, final_only, scale, b, h, rows):
-    """dQ for selected query rows of one (batch, query head); row-local."""
-    S, Hkv = k.shape[1], k.shape[2]
-    Hq = q.shape[2]
-    kh = h // (Hq // Hkv)
-    qpos_all = query_positions(S, n, final_only)
+def attn_bwd_dq_rows(q, k, v, do, n, mode, W, final_only, scale, b, h, rows, block=64):
+    """dQ for selected query rows of one (batch, query head); row-local:
+    dQ_i = scale sum_j P_ij (dO_i . V_j - dO_i . O_i) K_j."""
     rows = np.asarray(rows, dtype=np.int64)
     D = q.shape[-1]
     out = np.zeros((len(rows), D))
-    for i, r in enumerate(rows):
-        p = int(qpos_all[r])
-        lo = max(0, p - n * W + 1) if mode == CROSS_WINDOW else 0
-        keys = np.arange(lo, p + 1)
-        keys = keys[visible(p, keys, n, mode, W)]
-        kk = _f64(k[b, keys, kh, :])
-        vv = _f64(v[b, keys, kh, :])
-        qi = _f64(q[b, r, h, :])
-        doi = _f64(do[b, r, h, :])
-        sc = scale * (kk @ qi)
-        e = np.exp(sc - sc.max())
-        P = e / e.sum()
-        O = P @ vv
-        dP = vv @ doi
-        dS = P * (dP - doi @ O)
-        out[i] = scale * (dS @ kk)
+    for i in range(0, len(rows), block):
+        sel = rows[i:i + block]
+        _, K, V, P, _, _ = _row_block(q, k, v, n, mode, W, final_only, scale, b, h, sel)
+        dO = _f64(do[b, sel, h, :])
+        O = P @ V
+        dS = P * (dO @ V.T - (dO * O).sum(-1, keepdims=True))
+        out[i:i + block] = scale * (dS @ K)
     return out
 
 
-def attn_bwd_kv_cols(q, k, v, do, n, mode, W, final_only, scale, b, kh, cols):
+def attn_bwd_kv_cols(q, k, v, do, n, mode, W, final_only, scale, b, kh, cols, block=64):
     """dK, dV for selected key positions of one (batch, KV head).
 
     Every query that sees one of the keys gets its full row recomputed (LSE, O
@@ -227,31 +222,22 @@ def attn_bwd_kv_cols(q, k, v, do, n, mode, W, final_only, scale, b, kh, cols):
     D = q.shape[-1]
     cols = np.asarray(cols, dtype=np.int64)
     qpos_all = query_positions(S, n, final_only)
-    # queries that can see at least one selected key
-    mask_c = visible(qpos_all[:, None], cols[None, :], n, mode, W)
-    qrows = np.nonzero(mask_c.any(axis=1))[0]
+    sees = visible(qpos_all[:, None], cols[None, :], n, mode, W)
+    qrows = np.nonzero(sees.any(axis=1))[0]
     dk = np.zeros((len(cols), D))
     dv = np.zeros((len(cols), D))
-    kc = _f64(k[b, cols, kh, :])
     for h in range(kh * g, (kh + 1) * g):
-        for r in qrows:
-            p = int(qpos_all[r])
-            lo = max(0, p - n * W + 1) if mode == CROSS_WINDOW else 0
-            keys = np.arange(lo, p + 1)
-            keys = keys[visible(p, keys, n, mode, W)]
-            kk = _f64(k[b, keys, kh, :])
-            vv = _f64(v[b, keys, kh, :])
-            qi = _f64(q[b, r, h, :])
-            doi = _f64(do[b, r, h, :])
-            sc = scale * (kk @ qi)
-            mx = sc.max()
-            lse = mx + np.log(np.exp(sc - mx).sum())
-            O = np.exp(sc - lse) @ vv
-            Di = doi @ O
-            sel = mask_c[r]
-            pc = np.exp(scale * (kc[sel] @ qi) - lse)
-            dpc = _f64(v[b, cols[sel], kh, :]) @ doi
-            dsc = pc * (dpc - Di)
-            dk[sel] += scale * dsc[:, None] * qi[None, :]
-            dv[sel] += pc[:, None] * doi[None, :]
+        for i in range(0, len(qrows), block):
+            sel = qrows[i:i + block]
+            Q, K, V, P, _, lo = _row_block(q, k, v, n, mode, W, final_only, scale, b, h, sel)
+            dO = _f64(do[b, sel, h, :])
+            O = P @ V
+            Dvec = (dO * O).sum(-1)
+            # the selected keys inside this block's key window
+            inwin = (cols >= lo) & (cols < lo + K.shape[0])
+            idx = cols[inwin] - lo
+            Pc = P[:, idx]
+            dSc = Pc * (dO @ V[idx].T - Dvec[:, None])
+            dk[inwin] += scale * (dSc.T @ Q)
+            dv[inwin] += Pc.T @ dO
     return dk, dv

@@ -37,18 +37,19 @@ def decode_attn(q, k_cache, v_cache, seqlen, n, mode, W, scale):
     lse = np.zeros((B, Hq, n))
     for b in range(B):
         T = int(seqlen[b]) - 1
-        for s in range(n):
-            p = T * n + s
-            lo = max(0, p - n * W + 1) if mode == CROSS_WINDOW else 0
-            keys = np.arange(lo, p + 1)
-            keys = keys[visible(p, keys, n, mode, W)]
-            for kh in range(Hkv):
-                kk = _f64(k_cache[b, keys, kh, :])
-                vv = _f64(v_cache[b, keys, kh, :])
-                for h in range(kh * g, (kh + 1) * g):
-                    sc = scale * (kk @ q[b, s, h])
-                    mx = sc.max()
-                    e = np.exp(sc - mx)
-                    lse[b, h, s] = mx + np.log(e.sum())
-                    o[b, s, h] = (e / e.sum()) @ vv
+        qpos = T * n + np.arange(n)
+        lo = max(0, T * n - n * W + 1) if mode == CROSS_WINDOW else 0
+        keys = np.arange(lo, (T + 1) * n)
+        mask = visible(qpos[:, None], keys[None, :], n, mode, W)  # [n, keys]
+        for kh in range(Hkv):
+            kk = _f64(k_cache[b, lo:(T + 1) * n, kh, :])
+            vv = _f64(v_cache[b, lo:(T + 1) * n, kh, :])
+            for h in range(kh * g, (kh + 1) * g):
+                sc = scale * (q[b, :, h, :] @ kk.T)  # [n, keys]
+                sc = np.where(mask, sc, -np.inf)
+                mx = sc.max(axis=1, keepdims=True)
+                e = np.exp(sc - mx)
+                tot = e.sum(axis=1, keepdims=True)
+                lse[b, h, :] = (mx + np.log(tot))[:, 0]
+                o[b, :, h, :] = (e / tot) @ vv
     return o, lse

@@ -1,0 +1,166 @@
+/*
+ * hd.h - C ABI of the Hidden Decoding hot-path library (B200, sm_100a).
+ *
+ * The method (page "微信WeLM提出Hidden Decoding：大模型推理新范式", tahou.com):
+ *   - section "隐式序列缩放的技术细节", step 1: each token is expanded into n
+ *     streams; stream k of token i takes its input from the k-th of n embedding
+ *     tables and sits at physical position (i-1)n+k of an nL-long sequence.
+ *     0-based throughout this library: p = t*n + s, token(p) = p / n,
+ *     stream(p) = p % n.
+ *   - step 2: the expanded sequence runs through the unchanged Transformer with
+ *     causal attention and continuous positions (position encoding is applied
+ *     by the caller at the physical position p).
+ *   - section "规模化落地的工程优化": Stream-Factorized Attention. Intra-stream
+ *     layers see only earlier positions of the same stream; cross-stream layers
+ *     keep the base model's full-causal or sliding-window attention over the
+ *     whole expanded sequence. KV-mirror: only the final stream's queries pass
+ *     through the mirror layers and read K/V built for all n streams.
+ *   - section "实验效果与成本分析": at decode the n streams of a new token are
+ *     computed in one parallel step; the cache keeps K/V for every stream
+ *     (page "WeLM ...", aiflownews.com, "Latent computation scaling and Hidden
+ *     Decoding").
+ *
+ * Visibility rule (query at position p, key at position p'):
+ *   HD_INTRA        p' <= p  and  p' % n == p % n        (self included)
+ *   HD_CROSS_FULL   p' <= p
+ *   HD_CROSS_WINDOW p' <= p  and  p - p' < n * W_tokens  (W counted in tokens)
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer is DEVICE memory owned by the caller; tensors are dense and
+ *     row-major in the layouts stated below. "bf16" buffers hold IEEE bfloat16
+ *     bit patterns (2 bytes each). Pointers must be 16-byte aligned.
+ *   - The library allocates no memory and keeps no per-call state; scratch
+ *     space ("workspace") is passed in by the caller, sized by the matching
+ *     *_workspace_bytes() function.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream). Every call only enqueues work on that stream and returns.
+ *   - Argument errors are reported (HD_ERR_INVALID_ARG / HD_ERR_UNSUPPORTED)
+ *     before anything is launched. A failed launch returns HD_ERR_CUDA.
+ *     Errors found on the device (a token id outside the table, a bounded
+ *     wait that gave up) are recorded in a per-device status word, read and
+ *     cleared with hd_device_status(); kernels never trap.
+ */
+#ifndef HD_H_
+#define HD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HD_OK = 0,
+  HD_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, bad mode, ... */
+  HD_ERR_UNSUPPORTED = 2, /* valid arguments this build does not cover (e.g. D not in {64,128}) */
+  HD_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+  HD_ERR_TIMEOUT = 4,     /* device status: a bounded wait inside a kernel gave up */
+  HD_ERR_DEVICE_INDEX = 5 /* device status: a token id outside [0, V) (row left zero) */
+} hd_status;
+
+typedef enum { HD_INTRA = 0, HD_CROSS_FULL = 1, HD_CROSS_WINDOW = 2 } hd_mode;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* hd_status_string(int status);
+
+/* Library ABI version: (major << 16) | minor. */
+int hd_version(void);
+
+/*
+ * hd_expand_embed - interleaved n-table embedding gather.
+ * Source: tahou.com page, "隐式序列缩放的技术细节" step 1; aiflownews.com page,
+ * "Latent computation scaling and Hidden Decoding" (one table per stream).
+ *
+ *   out[b, t*n + s, :] = tables[s, ids[b, t], :]      (exact copy of the bytes)
+ *
+ *   ids     int32 [B, L]           token ids, must lie in [0, V)
+ *   tables  [n, V, d] elements of `elem_bytes` bytes (fp32: 4, bf16/fp16: 2)
+ *   out     [B, L*n, d] same element type
+ * An id outside [0, V) leaves its n output rows zero and records
+ * HD_ERR_DEVICE_INDEX in the device status word.
+ */
+int hd_expand_embed(const int32_t* ids, const void* tables, void* out, int B, int L, int n,
+                    int V, int d, int elem_bytes, void* stream);
+
+/*
+ * hd_attn_fwd - Stream-Factorized attention forward.
+ * Source: tahou.com page, "规模化落地的工程优化" (intra / cross-stream bullets,
+ * KV-mirror paragraph); "隐式序列缩放的技术细节" step 2 (causal attention).
+ *
+ *   O[p] = sum_{p' visible from p} softmax_p'(scale * q_p . k_p') v_p'
+ *   lse[p] = ln sum_{p' visible} exp(scale * q_p . k_p')
+ *
+ *   q    bf16 [B, S, Hq, D]   (S = n*L); with final_stream_queries_only:
+ *        bf16 [B, L, Hq, D], row t is the query at position t*n + n-1
+ *   k, v bf16 [B, S, Hkv, D]  (Hq % Hkv == 0; query head h reads KV head
+ *        h / (Hq/Hkv))
+ *   out  bf16, same shape as q
+ *   lse  fp32 [B, Hq, S] or [B, Hq, L] with final_stream_queries_only
+ *   mode hd_mode; W_tokens is the window in tokens (used by HD_CROSS_WINDOW
+ *        only, must be >= 1 there); scale is the softmax scale (> 0).
+ * Supported: D in {64, 128}. Accumulation is fp32; out is rounded to bf16.
+ */
+int hd_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int L,
+                int n, int Hq, int Hkv, int D, int mode, int W_tokens,
+                int final_stream_queries_only, float scale, void* stream);
+
+/* Bytes of workspace hd_attn_bwd needs for these sizes (0 on invalid sizes). */
+size_t hd_attn_bwd_workspace_bytes(int B, int L, int n, int Hq, int Hkv, int D,
+                                   int final_stream_queries_only);
+
+/*
+ * hd_attn_bwd - gradients of Stream-Factorized attention.
+ * Same source and arguments as hd_attn_fwd; out and lse are that call's
+ * outputs, dout has out's shape. Writes
+ *   dq (q's shape), dk, dv (k's shape), all bf16:
+ *   D_i = sum_d dO_id O_id, dP = dO V^T, dS = P * (dP - D),
+ *   dQ = scale dS K, dK = scale sum_{group} dS^T Q, dV = sum_{group} P^T dO.
+ * `workspace` must hold hd_attn_bwd_workspace_bytes(...) bytes of device
+ * memory (fp32 dQ accumulator and the D vector); its contents on entry do
+ * not matter and are overwritten.
+ */
+int hd_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                const void* dout, void* dq, void* dk, void* dv, int B, int L, int n, int Hq,
+                int Hkv, int D, int mode, int W_tokens, int final_stream_queries_only,
+                float scale, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace hd_decode_attn needs for these sizes (0 on invalid sizes). */
+size_t hd_decode_workspace_bytes(int B, int n, int Tcap, int Hq, int Hkv, int D);
+
+/*
+ * hd_decode_attn - one decode step of the n streams of a new token.
+ * Source: tahou.com page, "实验效果与成本分析" (the n streams are computed in
+ * one parallel forward; decode is bandwidth-bound at small batch) and
+ * "中间流的作用验证" (each stream keeps its own KV state).
+ *
+ *   q        bf16 [B, n, Hq, D]: the new token's n stream queries
+ *   k_cache, v_cache bf16 [B, Tcap*n, Hkv, D]: the expanded sequence in
+ *            position order. PRECONDITION: the new token's n K/V rows are
+ *            already written at positions T*n .. T*n+n-1, T = seqlen[b]-1.
+ *   seqlen   int32 [B] tokens per sequence INCLUDING the new one,
+ *            1 <= seqlen[b] <= Tcap (read on the device)
+ *   out      bf16 [B, n, Hq, D]; lse fp32 [B, Hq, n]
+ * Query s of sequence b sits at p = T*n + s and reads the cache positions
+ * the mode's visibility rule allows.
+ * `workspace` must hold hd_decode_workspace_bytes(...) bytes.
+ * A seqlen outside [1, Tcap] leaves that sequence's rows zero and records
+ * HD_ERR_DEVICE_INDEX in the device status word.
+ */
+int hd_decode_attn(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlen,
+                   void* out, float* lse, int B, int n, int Tcap, int Hq, int Hkv, int D, int mode,
+                   int W_tokens, float scale, void* workspace, size_t workspace_bytes,
+                   void* stream);
+
+/*
+ * Read (and, if `clear` is non-zero, reset) the device status word of the
+ * current device. Synchronizes `stream` first. Returns HD_OK when no kernel
+ * recorded an error since the last clear, else the first recorded code.
+ */
+int hd_device_status(void* stream, int clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HD_H_ */

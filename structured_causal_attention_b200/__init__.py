@@ -1,0 +1,117 @@
+"""Hidden Decoding hot path on B200: a C-ABI CUDA library and its Python binding.
+
+The library (``libhd.so``, built from ``csrc/`` by ``build.py``) implements the
+data-parallel hot path of Hidden Decoding with Stream-Factorized Attention
+(page "微信WeLM提出Hidden Decoding：大模型推理新范式", tahou.com):
+
+* ``hd_expand_embed``  interleaved n-table embedding gather (stream k of token i
+  at position (i-1)n+k);
+* ``hd_attn_fwd`` / ``hd_attn_bwd``  attention over the expanded sequence with
+  intra-stream, cross-stream full-causal and cross-stream sliding-window masks,
+  optionally with final-stream-only queries (KV-mirror);
+* ``hd_decode_attn``  the n stream queries of a new token against the
+  interleaved per-stream KV cache.
+
+The C names are re-exported from ``_lib`` (pointer + size arguments). The
+tensor helpers below (``expand_embed``, ``attn_fwd``, ``attn_bwd``,
+``decode_attn``) allocate outputs and workspace with torch and call the same C
+entry points; torch is used for device memory and streams only.
+"""
+from __future__ import annotations
+
+from ._lib import (  # noqa: F401
+    HD_ERR_CUDA,
+    HD_ERR_DEVICE_INDEX,
+    HD_ERR_INVALID_ARG,
+    HD_ERR_TIMEOUT,
+    HD_ERR_UNSUPPORTED,
+    HD_OK,
+    HDError,
+    hd_attn_bwd,
+    hd_attn_bwd_workspace_bytes,
+    hd_attn_fwd,
+    hd_decode_attn,
+    hd_decode_workspace_bytes,
+    hd_device_status,
+    hd_expand_embed,
+    lib,
+    status_string,
+)
+
+INTRA, CROSS_FULL, CROSS_WINDOW = 0, 1, 2
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensors must live on a CUDA device (the library has no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def expand_embed(ids, tables, stream=None):
+    """ids int32 [B, L], tables [n, V, d] -> out [B, L*n, d] (tables' dtype)."""
+    import torch
+
+    _need_cuda(ids, tables)
+    B, L = ids.shape
+    n, V, d = tables.shape
+    out = torch.empty((B, L * n, d), dtype=tables.dtype, device=tables.device)
+    hd_expand_embed(ids, tables, out, B, L, n, V, d, tables.element_size(), stream)
+    return out
+
+
+def attn_fwd(q, k, v, n, mode, W=0, final_only=False, scale=None, stream=None):
+    """q [B, Sq, Hq, D], k/v [B, n*L, Hkv, D] bf16 -> (out bf16 like q, lse fp32 [B, Hq, Sq])."""
+    import torch
+
+    _need_cuda(q, k, v)
+    B, S, Hkv, D = k.shape
+    L = S // n
+    Hq = q.shape[2]
+    if scale is None:
+        scale = D ** -0.5
+    out = torch.empty_like(q)
+    lse = torch.empty((B, Hq, q.shape[1]), dtype=torch.float32, device=q.device)
+    hd_attn_fwd(q, k, v, out, lse, B, L, n, Hq, Hkv, D, mode, W, final_only, scale, stream)
+    return out, lse
+
+
+def attn_bwd(q, k, v, out, lse, dout, n, mode, W=0, final_only=False, scale=None, stream=None,
+             workspace=None):
+    """Gradients (dq, dk, dv) in bf16; the fp32 workspace is allocated if not given."""
+    import torch
+
+    _need_cuda(q, k, v, out, lse, dout)
+    B, S, Hkv, D = k.shape
+    L = S // n
+    Hq = q.shape[2]
+    if scale is None:
+        scale = D ** -0.5
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    nbytes = hd_attn_bwd_workspace_bytes(B, L, n, Hq, Hkv, D, final_only)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    hd_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, L, n, Hq, Hkv, D, mode, W, final_only, scale,
+                workspace, workspace.numel() * workspace.element_size(), stream)
+    return dq, dk, dv
+
+
+def decode_attn(q, k_cache, v_cache, seqlen, mode, W=0, scale=None, stream=None, workspace=None):
+    """q [B, n, Hq, D]; caches [B, Tcap*n, Hkv, D]; seqlen int32 [B] (tokens incl. the new one)."""
+    import torch
+
+    _need_cuda(q, k_cache, v_cache, seqlen)
+    B, n, Hq, D = q.shape
+    Hkv = k_cache.shape[2]
+    Tcap = k_cache.shape[1] // n
+    if scale is None:
+        scale = D ** -0.5
+    out = torch.empty_like(q)
+    lse = torch.empty((B, Hq, n), dtype=torch.float32, device=q.device)
+    nbytes = hd_decode_workspace_bytes(B, n, Tcap, Hq, Hkv, D)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    hd_decode_attn(q, k_cache, v_cache, seqlen, out, lse, B, n, Tcap, Hq, Hkv, D, mode, W, scale,
+                   workspace, workspace.numel() * workspace.element_size(), stream)
+    return out, lse

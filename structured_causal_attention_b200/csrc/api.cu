@@ -1,0 +1,256 @@
+// api.cu - the C ABI declared in include/hd.h: argument validation, problem
+// set-up, launches. Everything is enqueued on the caller's stream; nothing is
+// allocated.
+#include <math.h>
+#include <mutex>
+
+#include "hd_common.cuh"
+#include "launch.h"
+
+namespace hd {
+
+// Per-device status word: kernels record the first error code here.
+__device__ int g_status_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices] = {};
+std::mutex g_status_mu;
+
+// Device address of the status word on the current device (looked up once per
+// device; host code must not pass the symbol itself to a kernel).
+int* status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_status_mu);
+  if (!g_status_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_status_word) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int*>(ptr);
+  }
+  return g_status_ptr[dev];
+}
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+constexpr long long kMaxPositions = 1LL << 28;  // positions and rows stay far below kWinInf
+
+int check_attn(const void* q, const void* k, const void* v, int B, int L, int n, int Hq, int Hkv,
+               int D, int mode, int W, int final_only, float scale) {
+  if (!q || !k || !v) return HD_ERR_INVALID_ARG;
+  if (B < 1 || L < 1 || n < 1 || Hq < 1 || Hkv < 1 || D < 1) return HD_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return HD_ERR_INVALID_ARG;
+  if (mode < HD_INTRA || mode > HD_CROSS_WINDOW) return HD_ERR_INVALID_ARG;
+  if (mode == HD_CROSS_WINDOW && W < 1) return HD_ERR_INVALID_ARG;
+  if (final_only != 0 && final_only != 1) return HD_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return HD_ERR_INVALID_ARG;
+  if (static_cast<long long>(n) * L > kMaxPositions) return HD_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return HD_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return HD_ERR_INVALID_ARG;
+  return HD_OK;
+}
+
+AttnParams make_params(const void* q, const void* k, const void* v, int B, int L, int n, int Hq,
+                       int Hkv, int D, int mode, int W, int final_only, float scale) {
+  AttnParams p = {};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.D = D;
+  p.n = n;
+  p.L = L;
+  p.S = n * L;
+  p.Sq = final_only ? L : n * L;
+  p.mode = mode;
+  p.final_only = final_only;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634074f;
+  p.status = status_ptr();
+  if (mode == HD_INTRA) {
+    // each stream is its own causal problem over the L tokens
+    p.groups = final_only ? 1 : n;
+    p.Lq = L;
+    p.Lk = L;
+    p.a = 1;
+    p.bb = 0;
+    p.win = kWinInf;
+    p.qs_step = final_only ? 0 : 1;
+    p.ks_step = final_only ? 0 : 1;
+    p.ks_base = final_only ? n - 1 : 0;
+    p.q_rstride = final_only ? 1 : n;
+    p.k_rstride = n;
+  } else {
+    p.groups = 1;
+    p.Lq = p.Sq;
+    p.Lk = p.S;
+    p.a = final_only ? n : 1;
+    p.bb = final_only ? n - 1 : 0;
+    const long long w = static_cast<long long>(n) * W;
+    p.win = (mode == HD_CROSS_WINDOW && w < p.S) ? static_cast<int>(w) : kWinInf;
+    p.qs_step = 0;
+    p.ks_step = 0;
+    p.ks_base = 0;
+    p.q_rstride = 1;
+    p.k_rstride = 1;
+  }
+  return p;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? HD_OK : HD_ERR_CUDA; }
+
+}  // namespace
+}  // namespace hd
+
+using namespace hd;
+
+extern "C" {
+
+const char* hd_status_string(int status) {
+  switch (status) {
+    case HD_OK: return "HD_OK";
+    case HD_ERR_INVALID_ARG: return "HD_ERR_INVALID_ARG: invalid argument";
+    case HD_ERR_UNSUPPORTED: return "HD_ERR_UNSUPPORTED: sizes not supported by this build";
+    case HD_ERR_CUDA: return "HD_ERR_CUDA: a CUDA call or launch failed";
+    case HD_ERR_TIMEOUT: return "HD_ERR_TIMEOUT: a bounded wait on the device gave up";
+    case HD_ERR_DEVICE_INDEX: return "HD_ERR_DEVICE_INDEX: an index read on the device was out of range";
+    default: return "unknown hd_status";
+  }
+}
+
+int hd_version(void) { return (1 << 16) | 0; }
+
+int hd_expand_embed(const int32_t* ids, const void* tables, void* out, int B, int L, int n, int V,
+                    int d, int elem_bytes, void* stream) {
+  if (!ids || !tables || !out) return HD_ERR_INVALID_ARG;
+  if (B < 1 || L < 1 || n < 1 || V < 1 || d < 1) return HD_ERR_INVALID_ARG;
+  if (elem_bytes != 1 && elem_bytes != 2 && elem_bytes != 4 && elem_bytes != 8)
+    return HD_ERR_INVALID_ARG;
+  const long long row_bytes = static_cast<long long>(d) * elem_bytes;
+  if (elem_bytes == 1 && row_bytes % 2 != 0) return HD_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(tables) | reinterpret_cast<uintptr_t>(out)) % 2 != 0)
+    return HD_ERR_INVALID_ARG;
+  return from_cuda(launch_expand(ids, tables, out, B, L, n, V, row_bytes, status_ptr(),
+                                 static_cast<cudaStream_t>(stream)));
+}
+
+int hd_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int L,
+                int n, int Hq, int Hkv, int D, int mode, int W_tokens,
+                int final_stream_queries_only, float scale, void* stream) {
+  int st = check_attn(q, k, v, B, L, n, Hq, Hkv, D, mode, W_tokens, final_stream_queries_only, scale);
+  if (st != HD_OK) return st;
+  if (!out || !lse || !aligned16(out)) return HD_ERR_INVALID_ARG;
+  AttnParams p = make_params(q, k, v, B, L, n, Hq, Hkv, D, mode, W_tokens,
+                             final_stream_queries_only, scale);
+  p.o = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  return from_cuda(launch_attn_fwd_mma(p, static_cast<cudaStream_t>(stream)));
+}
+
+size_t hd_attn_bwd_workspace_bytes(int B, int L, int n, int Hq, int Hkv, int D,
+                                   int final_stream_queries_only) {
+  if (B < 1 || L < 1 || n < 1 || Hq < 1 || Hkv < 1 || D < 1) return 0;
+  const size_t Sq = final_stream_queries_only ? static_cast<size_t>(L)
+                                              : static_cast<size_t>(n) * static_cast<size_t>(L);
+  const size_t rows = static_cast<size_t>(B) * Sq * static_cast<size_t>(Hq);
+  return align256(rows * static_cast<size_t>(D) * 4) + align256(rows * 4);
+}
+
+int hd_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                const void* dout, void* dq, void* dk, void* dv, int B, int L, int n, int Hq,
+                int Hkv, int D, int mode, int W_tokens, int final_stream_queries_only,
+                float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  int st = check_attn(q, k, v, B, L, n, Hq, Hkv, D, mode, W_tokens, final_stream_queries_only, scale);
+  if (st != HD_OK) return st;
+  if (!out || !lse || !dout || !dq || !dk || !dv || !workspace) return HD_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      !aligned16(workspace))
+    return HD_ERR_INVALID_ARG;
+  const size_t need = hd_attn_bwd_workspace_bytes(B, L, n, Hq, Hkv, D, final_stream_queries_only);
+  if (workspace_bytes < need) return HD_ERR_INVALID_ARG;
+  AttnParams p = make_params(q, k, v, B, L, n, Hq, Hkv, D, mode, W_tokens,
+                             final_stream_queries_only, scale);
+  p.o = static_cast<__nv_bfloat16*>(const_cast<void*>(out));
+  p.lse = const_cast<float*>(lse);
+  p.dout = static_cast<const __nv_bfloat16*>(dout);
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  const size_t rows = static_cast<size_t>(B) * p.Sq * Hq;
+  p.dq_acc = static_cast<float*>(workspace);
+  p.delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(rows * D * 4));
+  return from_cuda(launch_attn_bwd_mma(p, static_cast<cudaStream_t>(stream)));
+}
+
+size_t hd_decode_workspace_bytes(int B, int n, int Tcap, int Hq, int Hkv, int D) {
+  if (B < 1 || n < 1 || Tcap < 1 || Hq < 1 || Hkv < 1 || D < 1 || Hq % Hkv) return 0;
+  int mt = 0, splits = 0, chunk = 0;
+  decode_split_plan(B, n, Tcap, Hq, Hkv, &mt, &splits, &chunk);
+  const size_t prow = static_cast<size_t>(B) * Hkv * mt * 16 * splits;
+  return align256(prow * static_cast<size_t>(D) * 4) + align256(prow * 2 * 4);
+}
+
+int hd_decode_attn(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlen,
+                   void* out, float* lse, int B, int n, int Tcap, int Hq, int Hkv, int D, int mode,
+                   int W_tokens, float scale, void* workspace, size_t workspace_bytes,
+                   void* stream) {
+  if (!q || !k_cache || !v_cache || !seqlen || !out || !lse || !workspace) return HD_ERR_INVALID_ARG;
+  if (B < 1 || n < 1 || Tcap < 1 || Hq < 1 || Hkv < 1 || D < 1) return HD_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return HD_ERR_INVALID_ARG;
+  if (mode < HD_INTRA || mode > HD_CROSS_WINDOW) return HD_ERR_INVALID_ARG;
+  if (mode == HD_CROSS_WINDOW && W_tokens < 1) return HD_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return HD_ERR_INVALID_ARG;
+  if (static_cast<long long>(Tcap) * n > kMaxPositions) return HD_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return HD_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+      !aligned16(workspace))
+    return HD_ERR_INVALID_ARG;
+  const size_t need = hd_decode_workspace_bytes(B, n, Tcap, Hq, Hkv, D);
+  if (workspace_bytes < need) return HD_ERR_INVALID_ARG;
+  DecodeParams p = {};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.kc = static_cast<const __nv_bfloat16*>(k_cache);
+  p.vc = static_cast<const __nv_bfloat16*>(v_cache);
+  p.seqlen = seqlen;
+  p.o = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.status = status_ptr();
+  p.B = B;
+  p.n = n;
+  p.Tcap = Tcap;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.D = D;
+  p.mode = mode;
+  const long long w = static_cast<long long>(n) * W_tokens;
+  p.win = (mode == HD_CROSS_WINDOW && w < static_cast<long long>(Tcap) * n) ? static_cast<int>(w)
+                                                                           : kWinInf;
+  if (mode == HD_CROSS_WINDOW && p.win == kWinInf) p.mode = HD_CROSS_FULL;
+  p.rows = n * (Hq / Hkv);
+  decode_split_plan(B, n, Tcap, Hq, Hkv, &p.mt, &p.splits, &p.chunk);
+  const size_t prow = static_cast<size_t>(B) * Hkv * p.mt * 16 * p.splits;
+  p.part_o = static_cast<float*>(workspace);
+  p.part_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(prow * D * 4));
+  p.scale_log2 = scale * 1.4426950408889634074f;
+  return from_cuda(launch_decode(p, static_cast<cudaStream_t>(stream)));
+}
+
+int hd_device_status(void* stream, int clear) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return HD_ERR_CUDA;
+  int* ptr = status_ptr();
+  if (!ptr) return HD_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, ptr, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return HD_ERR_CUDA;
+  if (clear && v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(ptr, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return HD_ERR_CUDA;
+  }
+  return v;
+}
+
+}  // extern "C"

@@ -1,0 +1,39 @@
+// launch.h - internal host launchers (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "hd_common.cuh"
+
+namespace hd {
+
+constexpr int kWinInf = 1 << 30;  // "no window": larger than any supported sequence
+
+cudaError_t launch_attn_fwd_mma(const AttnParams& p, cudaStream_t stream);
+cudaError_t launch_attn_bwd_mma(const AttnParams& p, cudaStream_t stream);
+
+struct DecodeParams {
+  const __nv_bfloat16* q;   // [B, n, Hq, D]
+  const __nv_bfloat16* kc;  // [B, Tcap*n, Hkv, D]
+  const __nv_bfloat16* vc;
+  const int32_t* seqlen;    // [B]
+  __nv_bfloat16* o;         // [B, n, Hq, D]
+  float* lse;               // [B, Hq, n]
+  float* part_o;            // [B, Hkv, MT*16, splits, D] fp32
+  float* part_ml;           // [B, Hkv, MT*16, splits, 2] fp32 (max in log2 units, sum)
+  int* status;
+  int B, n, Tcap, Hq, Hkv, D, mode, win;  // win = n*W or kWinInf
+  int rows, mt, splits, chunk;             // rows = n*(Hq/Hkv); chunk keys per split
+  float scale_log2;
+};
+
+// Number of splits / chunk length the decode launcher uses for these sizes.
+void decode_split_plan(int B, int n, int Tcap, int Hq, int Hkv, int* mt, int* splits, int* chunk);
+cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
+
+cudaError_t launch_expand(const int32_t* ids, const void* tables, void* out, int B, int L, int n,
+                          int V, long long row_bytes, int* status, cudaStream_t stream);
+
+}  // namespace hd

@@ -1,0 +1,123 @@
+"""Forward parity: hd_attn_fwd (CUDA, through the C ABI) vs the float64 oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import structured_causal_attention_b200 as hd
+from structured_causal_attention_b200 import synthetic as syn
+from tests.gpu_util import LSE_MAX, O_MAX, O_MEAN, check, dev, host64, need_gpu, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+MODES = [hd.INTRA, hd.CROSS_FULL, hd.CROSS_WINDOW]
+
+
+def run_fwd(inp, n, mode, W, fin, scale):
+    q, k, v = dev(inp["q"]), dev(inp["k"]), dev(inp["v"])
+    out, lse = hd.attn_fwd(q, k, v, n, mode, W, fin, scale)
+    torch.cuda.synchronize()
+    assert hd.hd_device_status() == hd.HD_OK
+    return out, lse
+
+
+SMALL = [
+    # B, L, n, Hq, Hkv, D, W
+    (1, 64, 4, 4, 4, 64, 3),      # the tiny end-to-end case (+ a window)
+    (2, 37, 3, 4, 2, 128, 5),     # ragged L, GQA
+    (1, 50, 1, 2, 1, 64, 17),     # n = 1: textbook causal / sliding window
+    (1, 9, 8, 2, 2, 128, 2),      # n = 8, tiny L
+    (1, 1, 4, 2, 1, 64, 1),       # one token: S = n
+    (2, 130, 2, 6, 3, 64, 64),    # crosses a 128-row tile and a 64-key tile
+    (1, 200, 4, 2, 2, 128, 300),  # W > L (window = full causal)
+]
+
+
+@pytest.mark.parametrize("shape", SMALL, ids=[str(s) for s in SMALL])
+@pytest.mark.parametrize("mode", MODES, ids=["INTRA", "CROSS_FULL", "CROSS_WINDOW"])
+@pytest.mark.parametrize("fin", [0, 1], ids=["all", "final"])
+def test_fwd_small_full_compare(shape, mode, fin):
+    need_gpu()
+    B, L, n, Hq, Hkv, D, W = shape
+    scale = 1.0 / math.sqrt(D)
+    inp = syn.attention_inputs(B, L, n, Hq, Hkv, D, final_only=bool(fin), seed=L + n + D)
+    out, lse = run_fwd(inp, n, mode, W, fin, scale)
+    o_ref, l_ref = oracle.attn_fwd(inp["q"], inp["k"], inp["v"], n, mode, W, bool(fin), scale)
+    check(host64(out), o_ref, O_MAX, O_MEAN, "O")
+    check(host64(lse), l_ref, LSE_MAX, LSE_MAX, "LSE")
+
+
+def test_fwd_tiny_workload_exact_shapes():
+    """B1 L64 n4, 4 heads, D64, scale 1/8: INTRA and CROSS_FULL, every row."""
+    need_gpu()
+    w = syn.WORKLOADS["tiny"]
+    inp = syn.attention_inputs(w["B"], w["L"], w["n"], w["Hq"], w["Hkv"], w["D"], seed=1)
+    for mode in (hd.INTRA, hd.CROSS_FULL):
+        out, lse = run_fwd(inp, w["n"], mode, 0, 0, w["scale"])
+        o_ref, l_ref = oracle.attn_fwd(inp["q"], inp["k"], inp["v"], w["n"], mode, 1, False, w["scale"])
+        check(host64(out), o_ref, O_MAX, O_MEAN, "O")
+        check(host64(lse), l_ref, LSE_MAX, LSE_MAX, "LSE")
+
+
+def _sampled(name, mode, fin, seed, heads=None, rows_per_head=256):
+    need_gpu()
+    w = syn.WORKLOADS[name]
+    B, L, n, Hq, Hkv, D = w["B"], w["L"], w["n"], w["Hq"], w["Hkv"], w["D"]
+    W = w.get("W", 0)
+    inp = syn.attention_inputs(B, L, n, Hq, Hkv, D, final_only=fin, seed=seed)
+    out, lse = run_fwd(inp, n, mode, W, int(fin), w["scale"])
+    out_h, lse_h = out.cpu(), lse.cpu()
+    del out, lse
+    torch.cuda.empty_cache()
+    Sq = inp["q"].shape[1]
+    # float64 copies once per tensor; the oracle slices them per head
+    q64 = inp["q"].float().numpy().astype(np.float64)
+    k64 = inp["k"].float().numpy().astype(np.float64)
+    v64 = inp["v"].float().numpy().astype(np.float64)
+    pairs = [(b, h) for b in range(B) for h in range(Hq)] if heads is None else heads
+    errs = []
+    for (b, h) in pairs:
+        rows = sample_rows(Sq, n, W, fin, rows_per_head, seed * 1000 + b * 97 + h)
+        o_ref, l_ref = oracle.attn_fwd_rows(q64, k64, v64, n, mode, max(W, 1), fin, w["scale"], b, h, rows)
+        got_o = out_h[b, rows, h].float().numpy()
+        got_l = lse_h[b, h, rows].numpy()
+        errs.append(np.abs(got_o - o_ref))
+        check(got_l, l_ref, LSE_MAX, LSE_MAX, f"LSE b{b} h{h}")
+        assert np.abs(got_o - o_ref).max() <= O_MAX, (b, h)
+    allerr = np.concatenate([e.ravel() for e in errs])
+    assert allerr.mean() <= O_MEAN, allerr.mean()
+
+
+def test_fwd_intra_train_workload_sampled():
+    """B4, n4, L2048 (8192 positions), 16/4 heads, D128, INTRA; 256 rows per head."""
+    _sampled("intra_train", hd.INTRA, False, 2)
+
+
+def test_fwd_cross_window_workload_sampled():
+    """B2, n4, L8192, W=1024 tokens (4096 positions), 32/8 heads, D128; 256 rows per head."""
+    _sampled("cross_window", hd.CROSS_WINDOW, False, 3)
+
+
+def test_fwd_long_cross_full_workload_sampled():
+    """B1, n4, L32768 (131072 positions), 32/8 heads, D128, CROSS_FULL; 256 rows per head."""
+    _sampled("long_cross", hd.CROSS_FULL, False, 4)
+
+
+def test_fwd_long_final_stream_only_workload_sampled():
+    """KV-mirror: 32768 final-stream queries against all 131072 keys; 256 rows per head."""
+    _sampled("long_cross", hd.CROSS_FULL, True, 5)
+
+
+def test_fwd_final_only_matches_full_rows():
+    """Property at any size: final-only output equals the final-stream rows of the full run."""
+    need_gpu()
+    B, L, n, Hq, Hkv, D, W = 2, 300, 4, 8, 2, 128, 40
+    full = syn.attention_inputs(B, L, n, Hq, Hkv, D, seed=11)
+    for mode in MODES:
+        o_all, l_all = run_fwd(full, n, mode, W, 0, 0.09)
+        fin = {"q": full["q"][:, n - 1::n].contiguous(), "k": full["k"], "v": full["v"]}
+        o_fin, l_fin = run_fwd(fin, n, mode, W, 1, 0.09)
+        check(host64(o_fin), host64(o_all[:, n - 1::n]), 1e-2, 1e-4, "final rows")
+        check(host64(l_fin), host64(l_all[:, :, n - 1::n]), 1e-4, 1e-5, "final lse")

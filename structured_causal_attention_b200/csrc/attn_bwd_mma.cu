@@ -16,6 +16,8 @@
 //                 no atomics). dQ partials go to the fp32 accumulator with
 //                 vector atomics.
 //   3. bwd_dq:    dQ = bf16(scale * accumulator).
+// With INTRA and final-stream-only queries a fourth kernel zeroes the dK / dV
+// rows of streams 0..n-2, which no query reads.
 #include "hd_common.cuh"
 #include "launch.h"
 
@@ -65,6 +67,23 @@ __global__ void bwd_pre_kernel(const AttnParams p) {
   if (lane == 0) p.delta[(b * p.Hq + h) * p.Sq + i] = acc;
   float4* z = reinterpret_cast<float4*>(p.dq_acc + row * p.D);
   for (int c = lane; c < p.D / 4; c += 32) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// INTRA with final-stream-only queries: only stream n-1's keys are read, so
+// the dK / dV rows of streams 0..n-2 are exactly zero.
+__global__ void bwd_zero_unread_kv_kernel(const AttnParams p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long row = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + warp;  // (b, pos, hk)
+  const long long total = static_cast<long long>(p.B) * p.S * p.Hkv;
+  if (row >= total) return;
+  const long long pos = (row / p.Hkv) % p.S;
+  if (pos % p.n == p.n - 1) return;
+  uint2* zk = reinterpret_cast<uint2*>(p.dk + row * p.D);
+  uint2* zv = reinterpret_cast<uint2*>(p.dv + row * p.D);
+  for (int c = lane; c < p.D / 4; c += 32) {
+    zk[c] = make_uint2(0u, 0u);
+    zv[c] = make_uint2(0u, 0u);
+  }
 }
 
 __global__ void bwd_dq_kernel(const AttnParams p, long long n8) {
@@ -327,6 +346,12 @@ cudaError_t launch_bwd_d(const AttnParams& p, cudaStream_t stream) {
   bwd_main_kernel<D><<<static_cast<unsigned>(blocks), kBwdThreads, smem, stream>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (p.mode == HD_INTRA && p.final_only && p.n > 1) {
+    const long long kv_rows = static_cast<long long>(p.B) * p.S * p.Hkv;
+    bwd_zero_unread_kv_kernel<<<static_cast<unsigned>((kv_rows + 7) / 8), 256, 0, stream>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   const long long n8 = rows * D / 8;
   bwd_dq_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, stream>>>(p, n8);
   return cudaGetLastError();

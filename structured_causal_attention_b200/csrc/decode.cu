@@ -272,6 +272,9 @@ __global__ void decode_combine_kernel(const DecodeParams p) {
   float lt = 0.f;
   for (int j = 0; j < p.splits; ++j) {
     const float* ml = p.part_ml + (prow * p.splits + j) * 2;
+    // a chunk past the end of the sequence wrote only (max, sum) = (-inf, 0);
+    // its partial O was never written, so it must not be read
+    if (!(ml[1] > 0.f)) continue;
     const float f = fast_exp2(ml[0] - mu);
     lt += f * ml[1];
     const float* po = p.part_o + (prow * p.splits + j) * D;

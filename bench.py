@@ -291,6 +291,21 @@ def blas_threads():
         return os.cpu_count()
 
 
+# ------------------------------------------------------------------ ranks
+def reduce_max(values, device):
+    """Max over ranks of a list of floats (the timing rule for N > 1)."""
+    import torch.distributed as dist
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_value(flops_per_step, world, ms_per_step):
+    """Whole-job TFLOP/s: every rank runs its own replica of the step."""
+    return flops_per_step * max(world, 1) / (ms_per_step * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -418,14 +433,11 @@ def main():
     if hd.hd_device_status() != hd.HD_OK:
         raise RuntimeError("device status set during timing")
 
+    e2e_step = sum(e2e_ms) / len(e2e_ms)
     if world > 1:
-        t = torch.tensor([total_ms, sum(e2e_ms) / len(e2e_ms)], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_step = float(t[0]), float(t[1])
-    else:
-        e2e_step = sum(e2e_ms) / len(e2e_ms)
+        total_ms, e2e_step = reduce_max([total_ms, e2e_step], dev)
     ms_step = total_ms / args.steps
-    value = total_flops * max(world, 1) / (ms_step * 1e-3) / 1e12
+    value = whole_job_value(total_flops, world, ms_step)
 
     peaks = {}
     try:
@@ -459,7 +471,7 @@ def main():
         "data": "synthetic", "config": config,
         "expanded_tokens_per_s": round(tokens * max(world, 1) / (ms_step * 1e-3), 1),
         "decode_us_per_step": round(1e3 * dec["ms"], 2), "decode_gbs": dec.get("gbs"),
-        "e2e": {"value": round(total_flops * max(world, 1) / (e2e_step * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+        "e2e": {"value": round(whole_job_value(total_flops, world, e2e_step), 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": st.h2d_bytes, "d2h_bytes_per_step": st.d2h_bytes,
                 "ms_per_step": round(e2e_step, 4)},
         "gpu_launches": args.steps * sum(LAUNCHES[o["kind"]] for o in ops),

@@ -153,6 +153,33 @@ int hd_decode_attn(const void* q, const void* k_cache, const void* v_cache, cons
                    void* stream);
 
 /*
+ * hd_decode_attn_noalloc - hd_decode_attn for callers that cannot allocate.
+ * The pages have no counterpart: this is a deployment convenience.
+ *
+ * Some callers may not allocate device memory while they decode (a host
+ * framework that owns all GPU memory through its own pool, or a latency-bound
+ * loop that must not enter cudaMalloc, which can synchronise the device).
+ * This entry point takes the same arguments as hd_decode_attn minus the
+ * workspace, computes the same result, and keeps its split-K scratch in a
+ * fixed array of HD_DECODE_NOALLOC_SCRATCH_BYTES compiled into the library
+ * (held by every GPU that loads the library until the process exits). It
+ * allocates nothing and calls no allocating routine.
+ *   - Sizes whose hd_decode_workspace_bytes(...) exceeds
+ *     HD_DECODE_NOALLOC_SCRATCH_BYTES are rejected with HD_ERR_UNSUPPORTED.
+ *   - The first call on each device looks up the array's device address
+ *     (with that device current) and caches it; make that first call before
+ *     any stream capture.
+ *   - All calls on a device share the array, which keeps the last call's
+ *     contents; nothing in it needs to start at zero. Calls that overlap on
+ *     the GPU (two streams, or unordered host threads) race on it: order them.
+ */
+#define HD_DECODE_NOALLOC_SCRATCH_BYTES (16u << 20)
+int hd_decode_attn_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* seqlen, void* out, float* lse, int B, int n, int Tcap,
+                           int Hq, int Hkv, int D, int mode, int W_tokens, float scale,
+                           void* stream);
+
+/*
  * Read (and, if `clear` is non-zero, reset) the device status word of the
  * current device. Synchronizes `stream` first. Returns HD_OK when no kernel
  * recorded an error since the last clear, else the first recorded code.

@@ -31,6 +31,7 @@ from ._lib import (  # noqa: F401
     hd_attn_bwd_workspace_bytes,
     hd_attn_fwd,
     hd_decode_attn,
+    hd_decode_attn_noalloc,
     hd_decode_workspace_bytes,
     hd_device_status,
     hd_expand_embed,

@@ -36,6 +36,8 @@ SIGNATURES = {
     "hd_decode_workspace_bytes": (_Z, [_I, _I, _I, _I, _I, _I]),
     "hd_decode_attn": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _Z,
                             _P]),
+    "hd_decode_attn_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F,
+                                    _P]),
     "hd_device_status": (_I, [_P, _I]),
 }
 
@@ -127,6 +129,15 @@ def hd_decode_attn(q, k_cache, v_cache, seqlen, out, lse, B, n, Tcap, Hq, Hkv, D
                                        ptr(lse), B, n, Tcap, Hq, Hkv, D, mode, W_tokens, float(scale),
                                        ptr(workspace), int(workspace_bytes), stream_handle(stream)),
                   "hd_decode_attn")
+
+
+def hd_decode_attn_noalloc(q, k_cache, v_cache, seqlen, out, lse, B, n, Tcap, Hq, Hkv, D, mode,
+                           W_tokens, scale, stream=None):
+    """hd_decode_attn with the library's fixed scratch array (no workspace argument)."""
+    return _check(lib().hd_decode_attn_noalloc(ptr(q), ptr(k_cache), ptr(v_cache), ptr(seqlen),
+                                               ptr(out), ptr(lse), B, n, Tcap, Hq, Hkv, D, mode,
+                                               W_tokens, float(scale), stream_handle(stream)),
+                  "hd_decode_attn_noalloc")
 
 
 def hd_device_status(stream=None, clear=True):

@@ -149,7 +149,7 @@ int hd_attn_fwd(const void* q, const void* k, const void* v, void* out, float* l
                              final_stream_queries_only, scale);
   p.o = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
-  return from_cuda(launch_attn_fwd_mma(p, static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_attn_fwd_tc(p, static_cast<cudaStream_t>(stream)));
 }
 
 size_t hd_attn_bwd_workspace_bytes(int B, int L, int n, int Hq, int Hkv, int D,

@@ -11,7 +11,7 @@ namespace hd {
 
 constexpr int kWinInf = 1 << 30;  // "no window": larger than any supported sequence
 
-cudaError_t launch_attn_fwd_mma(const AttnParams& p, cudaStream_t stream);
+cudaError_t launch_attn_fwd_tc(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_attn_bwd_mma(const AttnParams& p, cudaStream_t stream);
 
 struct DecodeParams {

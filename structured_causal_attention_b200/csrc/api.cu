@@ -184,7 +184,7 @@ int hd_attn_bwd(const void* q, const void* k, const void* v, const void* out, co
   const size_t rows = static_cast<size_t>(B) * p.Sq * Hq;
   p.dq_acc = static_cast<float*>(workspace);
   p.delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(rows * D * 4));
-  return from_cuda(launch_attn_bwd_mma(p, static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_attn_bwd(p, static_cast<cudaStream_t>(stream)));
 }
 
 size_t hd_decode_workspace_bytes(int B, int n, int Tcap, int Hq, int Hkv, int D) {

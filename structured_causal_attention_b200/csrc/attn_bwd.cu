@@ -1,0 +1,99 @@
+// attn_bwd.cu - Stream-Factorized attention backward: launch sequence and the
+// small element-wise kernels around the tensor-core main kernel.
+//
+// Gradients of O = softmax(scale Q K^T over visible keys) V (page "微信WeLM提出
+// Hidden Decoding：大模型推理新范式", tahou.com, section "规模化落地的工程优化"):
+//   D_i = sum_d dO_id O_id,  P_ij = exp(scale q_i.k_j - LSE_i),
+//   dP = dO V^T,  dS = P * (dP - D),
+//   dQ = scale dS K,  dK = scale sum_group dS^T Q,  dV = sum_group P^T dO.
+//
+// Kernels on the caller's stream:
+//   1. bwd_pre:   D = rowsum(dO * O) (fp32, LSE layout); zero the fp32 dQ
+//                 accumulator.
+//   2. attn_bwd_tc_kernel (attn_bwd_tc.cu): dK, dV and the fp32 dQ sums.
+//   3. bwd_zero_unread_kv (INTRA with final-stream-only queries only): the dK /
+//                 dV rows of streams 0..n-2, which no query reads, are zero.
+//   4. bwd_dq:    dQ = bf16(scale * accumulator).
+#include "hd_common.cuh"
+#include "launch.h"
+
+namespace hd {
+
+namespace {
+
+__global__ void bwd_pre_kernel(const AttnParams p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long row = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + warp;
+  const long long total = static_cast<long long>(p.B) * p.Sq * p.Hq;
+  if (row >= total) return;
+  const int h = static_cast<int>(row % p.Hq);
+  const long long bi = row / p.Hq;
+  const long long i = bi % p.Sq, b = bi / p.Sq;
+  const __nv_bfloat16* o = p.o + row * p.D;
+  const __nv_bfloat16* g = p.dout + row * p.D;
+  float acc = 0.f;
+  for (int c = lane * 2; c < p.D; c += 64) {
+    const __nv_bfloat162 ov = *reinterpret_cast<const __nv_bfloat162*>(o + c);
+    const __nv_bfloat162 gv = *reinterpret_cast<const __nv_bfloat162*>(g + c);
+    acc = fmaf(__low2float(ov), __low2float(gv), acc);
+    acc = fmaf(__high2float(ov), __high2float(gv), acc);
+  }
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+  if (lane == 0) p.delta[(b * p.Hq + h) * p.Sq + i] = acc;
+  float4* z = reinterpret_cast<float4*>(p.dq_acc + row * p.D);
+  for (int c = lane; c < p.D / 4; c += 32) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// INTRA with final-stream-only queries: only stream n-1's keys are read, so
+// the dK / dV rows of streams 0..n-2 are exactly zero.
+__global__ void bwd_zero_unread_kv_kernel(const AttnParams p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long row = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + warp;  // (b, pos, hk)
+  const long long total = static_cast<long long>(p.B) * p.S * p.Hkv;
+  if (row >= total) return;
+  const long long pos = (row / p.Hkv) % p.S;
+  if (pos % p.n == p.n - 1) return;
+  uint2* zk = reinterpret_cast<uint2*>(p.dk + row * p.D);
+  uint2* zv = reinterpret_cast<uint2*>(p.dv + row * p.D);
+  for (int c = lane; c < p.D / 4; c += 32) {
+    zk[c] = make_uint2(0u, 0u);
+    zv[c] = make_uint2(0u, 0u);
+  }
+}
+
+__global__ void bwd_dq_kernel(const AttnParams p, long long n8) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const float4 a = reinterpret_cast<const float4*>(p.dq_acc)[2 * i];
+  const float4 c = reinterpret_cast<const float4*>(p.dq_acc)[2 * i + 1];
+  uint4 out;
+  out.x = pack_bf16(a.x * p.scale, a.y * p.scale);
+  out.y = pack_bf16(a.z * p.scale, a.w * p.scale);
+  out.z = pack_bf16(c.x * p.scale, c.y * p.scale);
+  out.w = pack_bf16(c.z * p.scale, c.w * p.scale);
+  reinterpret_cast<uint4*>(p.dq)[i] = out;
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bwd(const AttnParams& p, cudaStream_t stream) {
+  if (p.D != 64 && p.D != 128) return cudaErrorInvalidValue;
+  const long long rows = static_cast<long long>(p.B) * p.Sq * p.Hq;
+  bwd_pre_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = launch_attn_bwd_tc_main(p, stream);
+  if (e != cudaSuccess) return e;
+  if (p.mode == HD_INTRA && p.final_only && p.n > 1) {
+    const long long kv_rows = static_cast<long long>(p.B) * p.S * p.Hkv;
+    bwd_zero_unread_kv_kernel<<<static_cast<unsigned>((kv_rows + 7) / 8), 256, 0, stream>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  const long long n8 = rows * p.D / 8;
+  bwd_dq_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, stream>>>(p, n8);
+  return cudaGetLastError();
+}
+
+}  // namespace hd

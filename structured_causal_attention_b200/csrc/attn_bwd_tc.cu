@@ -1,0 +1,475 @@
+// attn_bwd_tc.cu - Stream-Factorized attention backward on tcgen05 + TMEM + TMA.
+//
+// Gradients of O = softmax(scale Q K^T over visible keys) V (page "微信WeLM提出
+// Hidden Decoding：大模型推理新范式", tahou.com, section "规模化落地的工程优化"):
+//   P_ij = exp(scale q_i.k_j - LSE_i), dP = dO V^T, dS = P * (dP - D),
+//   dQ = scale dS K,  dK = scale sum_group dS^T Q,  dV = sum_group P^T dO.
+//
+// One CTA owns 128 keys of one (batch, KV head, stream group) and loops over
+// the query heads of its GQA group and the 64-row query tiles that can see its
+// keys. Per query tile, on the tensor cores (one issuing thread, fp32 in TMEM):
+//   S^T  = K Q^T      (M 128 keys, N 64 queries)   } double-buffered in TMEM
+//   dP^T = V dO^T     (M 128 keys, N 64 queries)   }
+//   dV  += P^T dO     (M 128 keys, N D)            } accumulated in TMEM across
+//   dK  += dS^T Q     (M 128 keys, N D)            } the whole group
+//   dQ^T = K^T dS^T   (M D, N 64 queries)           into the S^T buffer
+// Roles (12 warps):
+//   warp 0      TMA: K, V once; Q and dO tiles (2 stages); its lanes also stage
+//               the tile's LSE and D values in shared memory.
+//   warp 1      TMEM allocation; lane 0 issues the MMAs.
+//   warps 4-7   one key row per thread: P^T = exp2(S^T - LSE), dS^T = P^T (dP^T - D),
+//               written as bf16 into shared memory in the MMA operand layout;
+//               at the end dK (scaled) and dV go out through TMA stores.
+//   warps 8-11  one head-dim row per thread: dQ^T from TMEM into an fp32 tile,
+//               added into the fp32 dQ accumulator with a TMA bulk reduce-add.
+// Every mbarrier wait is bounded (HD_ERR_TIMEOUT, then every role leaves).
+#include <cuda.h>
+
+#include "hd_common.cuh"
+#include "launch.h"
+#include "tc_ptx.cuh"
+
+namespace hd {
+
+namespace {
+
+constexpr int kKN = 128;   // keys per CTA
+constexpr int kQM = 64;    // query rows per iteration
+constexpr int kThreads = 384;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634074f;
+
+template <int D>
+struct BtSmem {
+  static constexpr int NSUB = D / 64;
+  static constexpr int KSUB = kKN * 128;    // [128 rows][64 bf16] sub-tile
+  static constexpr int QSUB = kQM * 128;    // [64 rows][64 bf16] sub-tile
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = K_OFF + NSUB * KSUB;
+  static constexpr int Q_OFF = V_OFF + NSUB * KSUB;          // 2 stages
+  static constexpr int DO_OFF = Q_OFF + 2 * NSUB * QSUB;     // 2 stages
+  static constexpr int P_OFF = DO_OFF + 2 * NSUB * QSUB;     // [128 keys][64 q] bf16
+  static constexpr int DS_OFF = P_OFF + kKN * 128;
+  static constexpr int DQ_OFF = DS_OFF + kKN * 128;          // D/32 boxes of [64 q][32] fp32
+  static constexpr int L_OFF = DQ_OFF + (D / 32) * kQM * 32 * 4;  // 2 stages x 64 LSE (log2)
+  static constexpr int DL_OFF = L_OFF + 2 * kQM * 4;              // 2 stages x 64 D
+  static constexpr int BAR_OFF = DL_OFF + 2 * kQM * 4;
+  static constexpr int NBAR = 15;
+  static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int ABORT_OFF = SLOT_OFF + 4;
+  static constexpr int USED = ABORT_OFF + 4 + 1024;
+  // at least 120 KB: one CTA (one 512-column TMEM allocation) per SM
+  static constexpr int TOTAL = USED > 120 * 1024 ? USED : 120 * 1024;
+};
+
+// barrier indices
+enum {
+  B_KV = 0,   // K and V loaded
+  B_QF = 1,   // [2] Q/dO (+ LSE, D) of a stage loaded: 1 tx arrival + 32 lane arrivals
+  B_QE = 3,   // [2] stage free (MMA commit)
+  B_SF = 5,   // [2] S^T / dP^T ready (MMA commit)
+  B_PF = 7,   // P^T / dS^T written (4 warp arrivals)
+  B_PE = 8,   // P^T / dS^T consumed by the MMAs (MMA commit)
+  B_DF = 9,   // [2] dQ^T ready (MMA commit)
+  B_DE = 11,  // [2] dQ^T read out (4 warp arrivals)
+  B_END = 13  // every MMA done (MMA commit)
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDK,
+                       const __grid_constant__ CUtensorMap tmDV, const __grid_constant__ CUtensorMap tmDQ) {
+  using SM = BtSmem<D>;
+  constexpr int NSUB = SM::NSUB;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
+  const uint32_t sK = sbase + SM::K_OFF, sV = sbase + SM::V_OFF, sQ = sbase + SM::Q_OFF,
+                 sDO = sbase + SM::DO_OFF, sP = sbase + SM::P_OFF, sDS = sbase + SM::DS_OFF,
+                 sDQ = sbase + SM::DQ_OFF;
+  float* sL = reinterpret_cast<float*>(sgen + SM::L_OFF);
+  float* sDl = reinterpret_cast<float*>(sgen + SM::DL_OFF);
+  auto bar = [&](int i) { return sbase + SM::BAR_OFF + 8u * i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + SM::ABORT_OFF);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (p.status && *reinterpret_cast<volatile int*>(p.status) == HD_ERR_TIMEOUT) return;
+
+  // ---- problem of this CTA: key tile kt of (b, hk, grp)
+  const int bkg = p.B * p.Hkv * p.groups;
+  const int kt = static_cast<int>(blockIdx.x / bkg);  // low key tiles see the most queries
+  int y = static_cast<int>(blockIdx.x % bkg);
+  const int grp = y % p.groups;
+  y /= p.groups;
+  const int hk = y % p.Hkv;
+  const int b = y / p.Hkv;
+  const int g = p.Hq / p.Hkv;
+  const bool intra = p.mode == HD_INTRA;
+  const int jk = intra ? (p.final_only ? p.n - 1 : grp) * p.Hkv + hk : hk;
+  const int c0 = kt * kKN;
+  const int c_last = min(c0 + kKN, p.Lk) - 1;
+  const int rmin = (c0 - p.bb <= 0) ? 0 : (c0 - p.bb + p.a - 1) / p.a;
+  const int rmax = min(p.Lq - 1, (c_last + p.win - 1 - p.bb) / p.a);
+  const int qt_lo = rmin / kQM;
+  const int nqt = rmin <= rmax ? rmax / kQM - qt_lo + 1 : 0;
+  const int total = g * nqt;
+  auto iter_head = [&](int it) { return hk * g + it / nqt; };
+  auto iter_row0 = [&](int it) { return (qt_lo + it % nqt) * kQM; };
+  auto jq_of = [&](int h) { return (intra && !p.final_only) ? grp * p.Hq + h : h; };
+
+  if (tid == 0) {
+    for (int i = 0; i < SM::NBAR; ++i) {
+      uint32_t cnt = 1;
+      if (i == B_QF || i == B_QF + 1) cnt = 33;
+      if (i == B_PF || i == B_DE || i == B_DE + 1) cnt = 4;
+      tc::mbar_init(bar(i), cnt);
+    }
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(sbase + SM::SLOT_OFF, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sgen + SM::SLOT_OFF);
+  // TMEM columns: buffer x in {0,1}: S^T at 128x, dP^T at 128x + 64 (dQ^T reuses S^T);
+  // dK at 256, dV at 256 + D.
+  const uint32_t tdK = tmem + 256, tdV = tmem + 256 + D;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tc::tma_prefetch_desc(&tmQ);
+      tc::tma_prefetch_desc(&tmDO);
+      tc::mbar_expect_tx(bar(B_KV), 2 * NSUB * SM::KSUB);
+#pragma unroll
+      for (int s = 0; s < NSUB; ++s) {
+        tc::tma_load_4d(sK + s * SM::KSUB, &tmK, bar(B_KV), s * 64, jk, c0, b);
+        tc::tma_load_4d(sV + s * SM::KSUB, &tmV, bar(B_KV), s * 64, jk, c0, b);
+      }
+    }
+    for (int it = 0; it < total; ++it) {
+      const int st = it & 1;
+      if (!tc::mbar_wait(bar(B_QE + st), ((it >> 1) & 1) ^ 1, abort_flag, p.status)) break;
+      const int h = iter_head(it), rq0 = iter_row0(it), jq = jq_of(h);
+      if (lane == 0) {
+        tc::mbar_expect_tx(bar(B_QF + st), 2 * NSUB * SM::QSUB);
+#pragma unroll
+        for (int s = 0; s < NSUB; ++s) {
+          tc::tma_load_4d(sQ + (st * NSUB + s) * SM::QSUB, &tmQ, bar(B_QF + st), s * 64, jq, rq0, b);
+          tc::tma_load_4d(sDO + (st * NSUB + s) * SM::QSUB, &tmDO, bar(B_QF + st), s * 64, jq, rq0, b);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int rr = lane + 32 * k, r = rq0 + rr;
+        float l2 = 0.f, dl = 0.f;
+        if (r < p.Lq) {
+          const long long li = (static_cast<long long>(b) * p.Hq + h) * p.Sq +
+                               static_cast<long long>(grp) * p.qs_step +
+                               static_cast<long long>(r) * p.q_rstride;
+          l2 = p.lse[li] * kLog2e;
+          dl = p.delta[li];
+        }
+        sL[st * kQM + rr] = l2;
+        sDl[st * kQM + rr] = dl;
+      }
+      tc::mbar_arrive(bar(B_QF + st));
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0 && total > 0) {
+      constexpr uint32_t idSP = tc::idesc_bf16_f32(128, kQM, 0, 0);  // S^T, dP^T
+      constexpr uint32_t idKV = tc::idesc_bf16_f32(128, D, 0, 1);    // dV, dK
+      constexpr uint32_t idDQ = tc::idesc_bf16_f32(128, kQM, 1, 1);  // dQ^T
+      // rows 64..127 of K^T for D = 64 read the V tile and are ignored
+      constexpr uint32_t kt_lbo = (D == 64) ? (SM::V_OFF - SM::K_OFF) : SM::KSUB;
+      auto issue_sp = [&](int buf, int st) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ko = (kk >> 2) * SM::KSUB + (kk & 3) * 32;
+          const uint32_t qo = (st * NSUB + (kk >> 2)) * SM::QSUB + (kk & 3) * 32;
+          tc::mma_ss(tmem + 128 * buf, tc::smem_desc_sw128(sK + ko, 16, 1024),
+                     tc::smem_desc_sw128(sQ + qo, 16, 1024), idSP, kk > 0);
+          tc::mma_ss(tmem + 128 * buf + 64, tc::smem_desc_sw128(sV + ko, 16, 1024),
+                     tc::smem_desc_sw128(sDO + qo, 16, 1024), idSP, kk > 0);
+        }
+      };
+      bool ok = tc::mbar_wait(bar(B_KV), 0, abort_flag, p.status) &&
+                tc::mbar_wait(bar(B_QF), 0, abort_flag, p.status);
+      if (ok) {
+        tc::tc_fence_after();
+        issue_sp(0, 0);
+        tc::mma_commit(bar(B_SF));
+      }
+      for (int it = 0; ok && it < total; ++it) {
+        const int x = it & 1, st = it & 1;
+        if (it + 1 < total) {
+          const int x1 = (it + 1) & 1;
+          ok = tc::mbar_wait(bar(B_QF + x1), ((it + 1) >> 1) & 1, abort_flag, p.status);
+          if (ok && it + 1 >= 2)
+            ok = tc::mbar_wait(bar(B_DE + x1), (((it + 1) >> 1) - 1) & 1, abort_flag, p.status);
+          if (!ok) break;
+          tc::tc_fence_after();
+          issue_sp(x1, x1);
+          tc::mma_commit(bar(B_SF + x1));
+        }
+        ok = tc::mbar_wait(bar(B_PF), it & 1, abort_flag, p.status);
+        if (!ok) break;
+        tc::tc_fence_after();
+        const uint32_t acc = it > 0 ? 1u : 0u;
+#pragma unroll
+        for (int kk = 0; kk < kQM / 16; ++kk) {  // reduce over the 64 queries
+          const uint64_t ap = tc::smem_desc_sw128(sP + kk * 32, 16, 1024);
+          const uint64_t as = tc::smem_desc_sw128(sDS + kk * 32, 16, 1024);
+          const uint64_t bo = tc::smem_desc_sw128(sDO + st * NSUB * SM::QSUB + kk * 2048, SM::QSUB, 1024);
+          const uint64_t bq = tc::smem_desc_sw128(sQ + st * NSUB * SM::QSUB + kk * 2048, SM::QSUB, 1024);
+          tc::mma_ss(tdV, ap, bo, idKV, (acc | kk) ? 1u : 0u);
+          tc::mma_ss(tdK, as, bq, idKV, (acc | kk) ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < kKN / 16; ++kk) {  // reduce over the 128 keys
+          const uint64_t ak = tc::smem_desc_sw128(sK + kk * 2048, kt_lbo, 1024);
+          const uint64_t bs = tc::smem_desc_sw128(sDS + kk * 2048, SM::QSUB, 1024);
+          tc::mma_ss(tmem + 128 * x, ak, bs, idDQ, kk > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(bar(B_DF + x));
+        tc::mma_commit(bar(B_QE + st));
+        tc::mma_commit(bar(B_PE));
+      }
+      tc::mma_commit(bar(B_END));
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------ P^T, dS^T (one key per thread)
+    const int row = tid - 128;
+    const int c = c0 + row;
+    const uint32_t tq = static_cast<uint32_t>((warp - 4) * 32) << 16;
+    bool ok = true;
+    for (int it = 0; it < total; ++it) {
+      const int x = it & 1, st = it & 1;
+      const int rq0 = iter_row0(it);
+      if (!tc::mbar_wait(bar(B_SF + x), (it >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+      tc::tc_fence_after();
+      const bool full = (c0 + kKN - 1 <= p.a * rq0 + p.bb) &&
+                        (c0 > p.a * (rq0 + kQM - 1) + p.bb - p.win) && (c0 + kKN <= p.Lk) &&
+                        (rq0 + kQM <= p.Lq);
+      if (it > 0) {
+        if (!tc::mbar_wait(bar(B_PE), (it - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+      }
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t sr[32], dr[32];
+        tc::tmem_ld32(tmem + tq + 128 * x + half * 32, sr);
+        tc::tmem_ld32(tmem + tq + 128 * x + 64 + half * 32, dr);
+        tc::tmem_wait_ld();
+        float pv[32], ds[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int rl = half * 32 + j;
+          const float l2 = sL[st * kQM + rl];
+          float pj = fast_exp2(fmaf(__uint_as_float(sr[j]), p.scale_log2, -l2));
+          if (!full) {
+            const int r = rq0 + rl;
+            const int hi = p.a * r + p.bb;
+            if (!(r < p.Lq && c <= hi && c > hi - p.win && c < p.Lk)) pj = 0.f;
+          }
+          pv[j] = pj;
+          ds[j] = pj * (__uint_as_float(dr[j]) - sDl[st * kQM + rl]);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int ch = half * 4 + k;
+          const uint32_t off = row * 128 + ((ch ^ (row & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(sP + off),
+                       "r"(pack_bf16(pv[8 * k], pv[8 * k + 1])), "r"(pack_bf16(pv[8 * k + 2], pv[8 * k + 3])),
+                       "r"(pack_bf16(pv[8 * k + 4], pv[8 * k + 5])), "r"(pack_bf16(pv[8 * k + 6], pv[8 * k + 7]))
+                       : "memory");
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(sDS + off),
+                       "r"(pack_bf16(ds[8 * k], ds[8 * k + 1])), "r"(pack_bf16(ds[8 * k + 2], ds[8 * k + 3])),
+                       "r"(pack_bf16(ds[8 * k + 4], ds[8 * k + 5])), "r"(pack_bf16(ds[8 * k + 6], ds[8 * k + 7]))
+                       : "memory");
+        }
+      }
+      tc::fence_async_smem();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar(B_PF));
+    }
+    // ---- dK (scaled), dV: TMEM -> bf16 -> shared memory (Q / dO stages) -> TMA store
+    if (ok && !*abort_flag && total > 0) ok = tc::mbar_wait(bar(B_END), 0, abort_flag, p.status);
+    if (ok && !*abort_flag) {
+      tc::tc_fence_after();
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const uint32_t src = t == 0 ? tdK : tdV;
+        const uint32_t dst = t == 0 ? sQ : sDO;  // 2 stages x NSUB x [64][64] = NSUB x [128][64]
+        const float sc = t == 0 ? p.scale : 1.f;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t v[32];
+          if (total > 0) {
+            tc::tmem_ld32(src + tq + cc * 32, v);
+            tc::tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0u;
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int d8 = cc * 4 + k;
+            const float* f = reinterpret_cast<const float*>(v + 8 * k);
+            const uint32_t addr = dst + (d8 >> 3) * SM::KSUB + row * 128 + (((d8 & 7) ^ (row & 7)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr),
+                         "r"(pack_bf16(f[0] * sc, f[1] * sc)), "r"(pack_bf16(f[2] * sc, f[3] * sc)),
+                         "r"(pack_bf16(f[4] * sc, f[5] * sc)), "r"(pack_bf16(f[6] * sc, f[7] * sc))
+                         : "memory");
+          }
+        }
+      }
+      tc::fence_async_smem();
+    }
+    asm volatile("bar.sync 1, 128;\n" ::: "memory");
+    if (row == 0 && ok && !*abort_flag) {
+#pragma unroll
+      for (int s = 0; s < NSUB; ++s) {
+        tc::tma_store_4d(&tmDK, sQ + s * SM::KSUB, s * 64, jk, c0, b);
+        tc::tma_store_4d(&tmDV, sDO + s * SM::KSUB, s * 64, jk, c0, b);
+      }
+      tc::tma_store_commit_and_wait();
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------- dQ^T readout (one head-dim row per thread)
+    const int d = tid - 256;
+    const uint32_t tq = static_cast<uint32_t>((warp - 8) * 32) << 16;
+    for (int it = 0; it < total; ++it) {
+      const int x = it & 1;
+      if (!tc::mbar_wait(bar(B_DF + x), (it >> 1) & 1, abort_flag, p.status)) break;
+      tc::tc_fence_after();
+      uint32_t v0[32], v1[32];
+      tc::tmem_ld32(tmem + tq + 128 * x, v0);
+      tc::tmem_ld32(tmem + tq + 128 * x + 32, v1);
+      tc::tmem_wait_ld();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar(B_DE + x));
+      // the previous reduce-add has finished reading the staging tile
+      if (d == 0) asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
+      asm volatile("bar.sync 2, 128;\n" ::: "memory");
+      if (d < D) {
+        float* stg = reinterpret_cast<float*>(sgen + SM::DQ_OFF) + (d >> 5) * (kQM * 32) + (d & 31);
+#pragma unroll
+        for (int q = 0; q < 32; ++q) stg[q * 32] = __uint_as_float(v0[q]);
+#pragma unroll
+        for (int q = 0; q < 32; ++q) stg[(q + 32) * 32] = __uint_as_float(v1[q]);
+      }
+      tc::fence_async_smem();
+      asm volatile("bar.sync 2, 128;\n" ::: "memory");
+      if (d == 0) {
+        const int h = iter_head(it), rq0 = iter_row0(it), jq = jq_of(h);
+#pragma unroll
+        for (int bx = 0; bx < D / 32; ++bx)
+          asm volatile(
+              "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group"
+              " [%0, {%2, %3, %4, %5}], [%1];\n" ::"l"(reinterpret_cast<uint64_t>(&tmDQ)),
+              "r"(sDQ + bx * kQM * 32 * 4), "r"(bx * 32), "r"(jq), "r"(rq0), "r"(b)
+              : "memory");
+        asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
+      }
+    }
+    if (d == 0) asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ----------------------------------------------------------------- host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// (d, j, row, batch) view; strides in elements; box (box_d, 1, box_rows, 1).
+bool make_map(CUtensorMap* map, const void* base, bool fp32, int D, long long J, long long R,
+              long long B, long long stride_j, long long stride_r, long long stride_b, int box_d,
+              int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const int es = fp32 ? 4 : 2;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(J),
+                              static_cast<cuuint64_t>(R), static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(stride_j * es),
+                                 static_cast<cuuint64_t>(stride_r * es),
+                                 static_cast<cuuint64_t>(stride_b * es)};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(box_d), 1, static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+            const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            fp32 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_bwd_tc_d(const AttnParams& p, cudaStream_t stream) {
+  const long long S = p.S, L = p.L, n = p.n, Hq = p.Hq, Hkv = p.Hkv, B = p.B;
+  CUtensorMap mq, mdo, mk, mv, mdk, mdv, mdq;
+  const bool intra = p.mode == HD_INTRA;
+  long long Jq, Rq, sjq, srq, sbq;
+  if (intra && !p.final_only) {
+    Jq = n * Hq; Rq = L; sjq = D; srq = n * Hq * D; sbq = S * Hq * D;
+  } else {
+    Rq = p.final_only ? L : S; Jq = Hq; sjq = D; srq = Hq * D; sbq = Rq * Hq * D;
+  }
+  long long Jk, Rk, srk, sbk;
+  if (intra) {
+    Jk = n * Hkv; Rk = L; srk = n * Hkv * D; sbk = S * Hkv * D;
+  } else {
+    Jk = Hkv; Rk = S; srk = Hkv * D; sbk = S * Hkv * D;
+  }
+  bool ok = make_map(&mq, p.q, false, D, Jq, Rq, B, sjq, srq, sbq, 64, kQM) &&
+            make_map(&mdo, p.dout, false, D, Jq, Rq, B, sjq, srq, sbq, 64, kQM) &&
+            make_map(&mdq, p.dq_acc, true, D, Jq, Rq, B, sjq, srq, sbq, 32, kQM) &&
+            make_map(&mk, p.k, false, D, Jk, Rk, B, D, srk, sbk, 64, kKN) &&
+            make_map(&mv, p.v, false, D, Jk, Rk, B, D, srk, sbk, 64, kKN) &&
+            make_map(&mdk, p.dk, false, D, Jk, Rk, B, D, srk, sbk, 64, kKN) &&
+            make_map(&mdv, p.dv, false, D, Jk, Rk, B, D, srk, sbk, 64, kKN);
+  if (!ok) return cudaErrorInvalidValue;
+  const int smem = BtSmem<D>::TOTAL;
+  cudaError_t e = cudaFuncSetAttribute(attn_bwd_tc_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const long long blocks = static_cast<long long>((p.Lk + kKN - 1) / kKN) * p.B * p.Hkv * p.groups;
+  attn_bwd_tc_kernel<D><<<static_cast<unsigned>(blocks), kThreads, smem, stream>>>(p, mq, mdo, mk, mv,
+                                                                                   mdk, mdv, mdq);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bwd_tc_main(const AttnParams& p, cudaStream_t stream) {
+  if (p.D == 64) return launch_bwd_tc_d<64>(p, stream);
+  if (p.D == 128) return launch_bwd_tc_d<128>(p, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace hd

@@ -12,7 +12,8 @@ namespace hd {
 constexpr int kWinInf = 1 << 30;  // "no window": larger than any supported sequence
 
 cudaError_t launch_attn_fwd_tc(const AttnParams& p, cudaStream_t stream);
-cudaError_t launch_attn_bwd_mma(const AttnParams& p, cudaStream_t stream);
+cudaError_t launch_attn_bwd(const AttnParams& p, cudaStream_t stream);
+cudaError_t launch_attn_bwd_tc_main(const AttnParams& p, cudaStream_t stream);
 
 struct DecodeParams {
   const __nv_bfloat16* q;   // [B, n, Hq, D]

@@ -92,62 +92,115 @@ def step_plan(wl):
 
 LAUNCHES = {"expand": 1, "fwd": 1, "bwd": 3, "decode": 2}
 
+# Extra workloads for per-configuration measurements (`--workload`); the
+# default is the whole hot-path step above.
+WORKLOADS = {
+    "step": dict(WL, ops=None),
+    "intra_train": dict(B=4, L=2048, n=4, Hq=16, Hkv=4, D=128, W=1024, V=32000, d=2048, T=2048,
+                        ops=["fwd_intra", "bwd_intra"]),
+    "cross_window": dict(B=2, L=8192, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=8192,
+                         ops=["fwd_cross_window", "bwd_cross_window"]),
+    "long_cross": dict(B=1, L=32768, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=32768,
+                       ops=["fwd_cross_full", "fwd_final_only"]),
+    "decode8": dict(B=8, L=1, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=16384,
+                    ops=["decode_cross_full", "decode_intra"]),
+    "decode64": dict(B=64, L=1, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=16384,
+                     ops=["decode_cross_full", "decode_intra"]),
+    "expand": dict(B=4, L=8192, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=1,
+                   ops=["expand"]),
+}
+
+
+def plan_for(name):
+    wl = dict(WORKLOADS[name])
+    ops = step_plan(wl)
+    if wl["ops"] is not None:
+        ops = [o for o in ops if o["name"] in wl["ops"]]
+    return wl, ops
+
 
 # --------------------------------------------------------------- GPU state
 class Step:
-    """Device buffers of one step plus the calls that make up the step."""
+    """Device buffers of one step plus the calls that make up the step.
 
-    def __init__(self, wl, dev):
+    Only the buffers the step's operations use are allocated.
+    """
+
+    def __init__(self, wl, ops, dev):
         import structured_causal_attention_b200 as hd
         from structured_causal_attention_b200 import synthetic as syn
 
         self.hd, self.wl, self.dev = hd, wl, dev
         B, n, L, Hq, Hkv, D, V, d, T = (wl[k] for k in ("B", "n", "L", "Hq", "Hkv", "D", "V", "d", "T"))
         S = n * L
-        self.S = S
+        kinds = {o["kind"] for o in ops}
+        names = {o["name"] for o in ops}
+        attn = kinds & {"fwd", "bwd"}
+        fin = any(o.get("fin") for o in ops if o["kind"] in ("fwd", "bwd"))
+        full = any(not o.get("fin") for o in ops if o["kind"] in ("fwd", "bwd"))
         # host copies (pinned) of every per-step input, for the end-to-end leg
-        a = syn.attention_inputs(B, L, n, Hq, Hkv, D, seed=2, with_grad=True)
-        self.h = {
-            "ids": syn.token_ids(B, L, V, seed=9),
-            "q": a["q"], "k": a["k"], "v": a["v"], "do": a["do"],
-            "qf": syn.normal_bf16((B, L, Hq, D), 12),
-            "dof": syn.normal_bf16((B, L, Hq, D), 13),
-            "dq_new": syn.normal_bf16((B, n, Hq, D), 14),
-        }
+        self.h = {}
+        if "expand" in kinds:
+            self.h["ids"] = syn.token_ids(B, L, V, seed=9)
+        if attn:
+            a = syn.attention_inputs(B, L, n, Hq, Hkv, D, seed=2, with_grad="bwd" in kinds)
+            self.h.update({"k": a["k"], "v": a["v"]})
+            if full:
+                self.h["q"] = a["q"]
+                if "bwd" in kinds:
+                    self.h["do"] = a["do"]
+            if fin:
+                self.h["qf"] = syn.normal_bf16((B, L, Hq, D), 12)
+                if "bwd" in kinds:
+                    self.h["dof"] = syn.normal_bf16((B, L, Hq, D), 13)
+        if "decode" in kinds:
+            self.h["dq_new"] = syn.normal_bf16((B, n, Hq, D), 14)
         for k_ in list(self.h):
             self.h[k_] = self.h[k_].pin_memory()
         self.d = {k_: v_.to(dev) for k_, v_ in self.h.items()}
-        # model state kept resident: embedding tables and the KV cache
         g = torch.Generator(device=dev)
         g.manual_seed(15)
-        self.tables = torch.empty((n, V, d), dtype=torch.float32, device=dev).normal_(0, 0.02, generator=g)
-        self.kc = torch.empty((B, (T + 1) * n, Hkv, D), dtype=torch.bfloat16, device=dev).normal_(generator=g)
-        self.vc = torch.empty_like(self.kc).normal_(generator=g)
-        self.seqlen = torch.full((B,), T + 1, dtype=torch.int32, device=dev)
-        # outputs and workspaces
-        self.x = torch.empty((B, S, d), dtype=torch.float32, device=dev)
-        self.o = {m: torch.empty_like(self.d["q"]) for m in ("intra", "cross_full", "cross_window")}
-        self.lse = {m: torch.empty((B, Hq, S), dtype=torch.float32, device=dev)
-                    for m in ("intra", "cross_full", "cross_window")}
-        self.o["final_only"] = torch.empty_like(self.d["qf"])
-        self.lse["final_only"] = torch.empty((B, Hq, L), dtype=torch.float32, device=dev)
-        self.dq = torch.empty_like(self.d["q"])
-        self.dk = torch.empty_like(self.d["k"])
-        self.dv = torch.empty_like(self.d["v"])
-        self.dqf = torch.empty_like(self.d["qf"])
-        self.ws_bwd_n = hd.hd_attn_bwd_workspace_bytes(B, L, n, Hq, Hkv, D, 0)
-        self.ws_bwd = torch.empty(self.ws_bwd_n, dtype=torch.uint8, device=dev)
-        self.ws_dec_n = hd.hd_decode_workspace_bytes(B, n, T + 1, Hq, Hkv, D)
-        self.ws_dec = torch.empty(self.ws_dec_n, dtype=torch.uint8, device=dev)
-        self.dec_o = {m: torch.empty_like(self.d["dq_new"]) for m in ("cross_full", "intra")}
-        self.dec_l = {m: torch.empty((B, Hq, n), dtype=torch.float32, device=dev) for m in ("cross_full", "intra")}
+        # model state kept resident: embedding tables and the KV cache
+        if "expand" in kinds:
+            self.tables = torch.empty((n, V, d), dtype=torch.float32, device=dev).normal_(0, 0.02, generator=g)
+            self.x = torch.empty((B, S, d), dtype=torch.float32, device=dev)
+        if "decode" in kinds:
+            self.kc = torch.empty((B, (T + 1) * n, Hkv, D), dtype=torch.bfloat16, device=dev).normal_(generator=g)
+            self.vc = torch.empty_like(self.kc).normal_(generator=g)
+            self.seqlen = torch.full((B,), T + 1, dtype=torch.int32, device=dev)
+            self.ws_dec_n = hd.hd_decode_workspace_bytes(B, n, T + 1, Hq, Hkv, D)
+            self.ws_dec = torch.empty(self.ws_dec_n, dtype=torch.uint8, device=dev)
+            self.dec_o = {m: torch.empty_like(self.d["dq_new"]) for m in ("cross_full", "intra")}
+            self.dec_l = {m: torch.empty((B, Hq, n), dtype=torch.float32, device=dev)
+                          for m in ("cross_full", "intra")}
+        self.o, self.lse = {}, {}
+        for o in ops:
+            if o["kind"] == "fwd":
+                key = o["name"].split("_", 1)[1]
+                rows = L if o["fin"] else S
+                self.o[key] = torch.empty((B, rows, Hq, D), dtype=torch.bfloat16, device=dev)
+                self.lse[key] = torch.empty((B, Hq, rows), dtype=torch.float32, device=dev)
+        if "bwd" in kinds:
+            if full:
+                self.dq = torch.empty_like(self.d["q"])
+            if fin:
+                self.dqf = torch.empty_like(self.d["qf"])
+            self.dk = torch.empty_like(self.d["k"])
+            self.dv = torch.empty_like(self.d["v"])
+            self.ws_bwd_n = hd.hd_attn_bwd_workspace_bytes(B, L, n, Hq, Hkv, D, 0 if full else 1)
+            self.ws_bwd = torch.empty(self.ws_bwd_n, dtype=torch.uint8, device=dev)
         self.flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
         self.h2d_bytes = sum(t.numel() * t.element_size() for t in self.h.values())
-        self.d2h_bytes = sum(t.numel() * t.element_size() for t in self.dec_o.values()) + \
-            self.lse["intra"].numel() * 4
-        self.host_out = {m: torch.empty(self.dec_o[m].shape, dtype=self.dec_o[m].dtype).pin_memory()
-                         for m in self.dec_o}
-        self.host_lse = torch.empty(self.lse["intra"].shape, dtype=torch.float32).pin_memory()
+        # the step's result read back to the host: decode outputs, else the first forward's LSE
+        self.result = []
+        if "decode" in kinds:
+            self.result += list(self.dec_o.values())
+        elif self.lse:
+            self.result.append(next(iter(self.lse.values())))
+        elif "expand" in kinds:
+            self.result.append(self.x[:, :1])
+        self.host_res = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in self.result]
+        self.d2h_bytes = sum(t.numel() * t.element_size() for t in self.result)
 
     def call(self, op, stream):
         hd, wl, d = self.hd, self.wl, self.d
@@ -161,11 +214,11 @@ class Step:
             key = name.split("_", 1)[1]
             fin = op["fin"]
             q = d["qf"] if fin else d["q"]
-            do = d["dof"] if fin else d["do"]
             if op["kind"] == "fwd":
                 hd.hd_attn_fwd(q, d["k"], d["v"], self.o[key], self.lse[key], B, L, n, Hq, Hkv, D,
                                op["mode"], W, fin, sc, s)
             else:
+                do = d["dof"] if fin else d["do"]
                 hd.hd_attn_bwd(q, d["k"], d["v"], self.o[key], self.lse[key], do,
                                self.dqf if fin else self.dq, self.dk, self.dv, B, L, n, Hq, Hkv, D,
                                op["mode"], W, fin, sc, self.ws_bwd, self.ws_bwd_n, s)
@@ -180,9 +233,8 @@ class Step:
             self.d[k_].copy_(v_, non_blocking=True)
 
     def d2h(self, stream):
-        for m in self.dec_o:
-            self.host_out[m].copy_(self.dec_o[m], non_blocking=True)
-        self.host_lse.copy_(self.lse["intra"], non_blocking=True)
+        for h_, t_ in zip(self.host_res, self.result):
+            h_.copy_(t_, non_blocking=True)
 
 
 # ------------------------------------------------------------------ clocks
@@ -243,10 +295,9 @@ class ClockSampler:
 def oracle_sample(budget_s, wl, seed=0):
     """Time the float64 oracle on a bounded sample of the step's attention work.
 
-    Returns (unmasked FLOPs done, seconds, description). Rows are drawn from
-    every attention operation of the step, forward (4*D per pair) and dQ of
-    the backward (counted at the same 4*D the oracle spends per dQ pair is not
-    claimed: only forward FLOPs are credited).
+    Returns (unmasked FLOPs done, seconds, description). Query rows are drawn
+    from the four forward operations of the step (INTRA, CROSS_FULL,
+    CROSS_WINDOW, final-stream-only) and credited 4*D FLOPs per visible pair.
     """
     import oracle
     from structured_causal_attention_b200 import synthetic as syn
@@ -307,30 +358,48 @@ def whole_job_value(flops_per_step, world, ms_per_step):
 
 
 # ------------------------------------------------------------------- main
+DESCRIPTIONS = {
+    "step": "intra_train-sized hot-path step: B4 n4 L2048 (8192 expanded positions), Hq16 Hkv4 D128; "
+            "expand (V32000 d2048 fp32 tables) + fwd/bwd INTRA, CROSS_FULL, CROSS_WINDOW(W=1024 tokens), "
+            "final-stream-only + decode (cache 2048 tokens, CROSS_FULL and INTRA)",
+    "intra_train": "INTRA fwd+bwd, B4 n4 L2048 (8192 expanded), Hq16 Hkv4 D128",
+    "cross_window": "CROSS_WINDOW fwd+bwd, B2 n4 L8192 (32768 expanded), W=1024 tokens, Hq32 Hkv8 D128",
+    "long_cross": "CROSS_FULL fwd (131072 queries) + final-stream-only fwd (32768 queries), B1 n4 L32768, "
+                  "Hq32 Hkv8 D128",
+    "decode8": "decode step CROSS_FULL + INTRA, B8 n4, 16384 prior tokens (65540 cache rows), Hq32 Hkv8 D128",
+    "decode64": "decode step CROSS_FULL + INTRA, B64 n4, 16384 prior tokens (65540 cache rows), Hq32 Hkv8 D128",
+    "expand": "expansion B4 L8192 n4, V32000, d4096 fp32 tables",
+}
+
+# DRAM bytes per launch of the dominant kernel from the last ncu capture of
+# the same build (dram__bytes_read.sum + dram__bytes_write.sum); None when the
+# kernel changed after that capture.
+NCU_TRAFFIC = {}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="step", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    wl = dict(WL)
-    ops = step_plan(wl)
+    wl, ops = plan_for(args.workload)
     total_flops = sum(o["flops"] for o in ops)
+    total_bytes = sum(o.get("bytes", 0) for o in ops)
+    hbm_only = total_flops == 0 or all(o["kind"] in ("decode", "expand") for o in ops)
     tokens = wl["B"] * wl["n"] * wl["L"]
-    config = {"workload": "intra_train-sized hot-path step: B4 n4 L2048 (8192 expanded positions), "
-                          "Hq16 Hkv4 D128; expand (V32000 d2048 fp32 tables) + fwd/bwd INTRA, "
-                          "CROSS_FULL, CROSS_WINDOW(W=1024 tokens), final-stream-only + decode "
-                          "(cache 2048 tokens, CROSS_FULL and INTRA)",
+    config = {"workload": DESCRIPTIONS[args.workload],
               "global_batch": wl["B"] * max(world, 1), "seq_len": wl["n"] * wl["L"],
               "parallelism": f"replicas{max(world, 1)}",
               "l2": "256 MB buffer written between timed steps (outside the per-step events); "
-                    "per-step working set > 1 GB"}
+                    "per-step working set larger than L2"}
 
     if args.impl == "reference":
         if rank != 0:
@@ -338,7 +407,7 @@ def main():
         budget = 2.0
         vals = []
         for i in range(args.warmup + args.steps):
-            fl, dt, desc = oracle_sample(budget, wl, seed=i)
+            fl, dt, desc = oracle_sample(budget, WORKLOADS["step"], seed=i)
             if i >= args.warmup:
                 vals.append((fl, dt))
         fl = sum(v[0] for v in vals)
@@ -373,7 +442,7 @@ def main():
     import structured_causal_attention_b200 as hd
 
     hd.lib()
-    st = Step(wl, dev)
+    st = Step(wl, ops, dev)
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
 
@@ -437,7 +506,6 @@ def main():
     if world > 1:
         total_ms, e2e_step = reduce_max([total_ms, e2e_step], dev)
     ms_step = total_ms / args.steps
-    value = whole_job_value(total_flops, world, ms_step)
 
     peaks = {}
     try:
@@ -459,31 +527,53 @@ def main():
             rec["gbs"] = round(op["bytes"] / (m * 1e-3) / 1e9, 1)
             rec["frac_of_measured_hbm"] = round(rec["gbs"] / hbm_peak, 4)
         per_op[op["name"]] = rec
-    dom = max((o for o in ops if o["kind"] in ("fwd", "bwd")), key=lambda o: per_op[o["name"]]["ms"])
+    dom = max(ops, key=lambda o: per_op[o["name"]]["ms"])
     dom_ms = per_op[dom["name"]]["ms"]
-    ach = dom["flops"] / (dom_ms * 1e-3) / 1e12
-    traffic = None
-    dec = per_op["decode_cross_full"]
+    if dom["kind"] in ("fwd", "bwd"):
+        ach = dom["flops"] / (dom_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": tf_peak, "unit": "TFLOP/s",
+                "frac": round(ach / tf_peak, 4),
+                "peak_source": "MEASURED_PEAKS.json bf16_tflops_sustained" if peaks else "fallback 1400"}
+    else:
+        ach = dom["bytes"] / (dom_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(ach / hbm_peak, 4),
+                "peak_source": "MEASURED_PEAKS.json hbm_gbs" if peaks else "fallback 6650"}
+    kname = {"fwd": "hd_attn_fwd (attn_fwd_tc_kernel)",
+             "bwd": "hd_attn_bwd (bwd_pre + attn_bwd_tc_kernel + bwd_dq)",
+             "decode": "hd_decode_attn (decode_split + decode_combine)",
+             "expand": "hd_expand_embed (expand_kernel)"}[dom["kind"]]
+    roof = {"kernel": f"{kname}, op {dom['name']}", **roof,
+            "traffic": NCU_TRAFFIC.get((args.workload, dom["name"]))}
+    if hbm_only:
+        value = total_bytes * max(world, 1) / (ms_step * 1e-3) / 1e9
+        e2e_val = total_bytes * max(world, 1) / (e2e_step * 1e-3) / 1e9
+        unit = "GB/s"
+    else:
+        value = whole_job_value(total_flops, world, ms_step)
+        e2e_val = whole_job_value(total_flops, world, e2e_step)
+        unit = "TFLOP/s"
     out = {
-        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": max(world, 1),
+        "metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": max(world, 1),
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": config,
-        "expanded_tokens_per_s": round(tokens * max(world, 1) / (ms_step * 1e-3), 1),
-        "decode_us_per_step": round(1e3 * dec["ms"], 2), "decode_gbs": dec.get("gbs"),
-        "e2e": {"value": round(whole_job_value(total_flops, world, e2e_step), 2), "unit": "TFLOP/s",
+        "e2e": {"value": round(e2e_val, 2), "unit": unit,
                 "h2d_bytes_per_step": st.h2d_bytes, "d2h_bytes_per_step": st.d2h_bytes,
                 "ms_per_step": round(e2e_step, 4)},
         "gpu_launches": args.steps * sum(LAUNCHES[o["kind"]] for o in ops),
-        "roofline": {"kernel": f"hd_attn_{dom['kind']} ({dom['name']})", "bound": "tensor",
-                     "achieved": round(ach, 1), "peak": tf_peak, "unit": "TFLOP/s",
-                     "frac": round(ach / tf_peak, 4), "traffic": traffic,
-                     "peak_source": "MEASURED_PEAKS.json bf16_tflops_sustained" if peaks else "fallback"},
+        "roofline": roof,
         "per_op": per_op,
         "clocks": clocks,
     }
+    if tokens and not hbm_only:
+        out["expanded_tokens_per_s"] = round(tokens * max(world, 1) / (ms_step * 1e-3), 1)
+    dec = per_op.get("decode_cross_full")
+    if dec:
+        out["decode_us_per_step"] = round(1e3 * dec["ms"], 2)
+        out["decode_gbs"] = dec.get("gbs")
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        fl, dt, desc = oracle_sample(10.0, wl)
+        fl, dt, desc = oracle_sample(10.0, WORKLOADS["step"])
         out["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
                                "kind": "oracle", "sample": f"{dt:.1f} s: " + desc}
     if world > 1:

@@ -102,6 +102,17 @@ AttnParams make_params(const void* q, const void* k, const void* v, int B, int L
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+size_t pad64(size_t x) { return (x + 63) / 64 * 64; }
+
+// Rows of the packed per-problem statistics (LSE, D) for any mode: each
+// problem's rows are padded to a multiple of 64.
+size_t packed_rows(int B, int L, int n, int Hq, int final_only) {
+  // n * pad64(L) >= pad64(n * L): covers the n INTRA streams and the single
+  // cross-stream problem alike
+  const size_t per_bh = final_only ? pad64(L) : static_cast<size_t>(n) * pad64(L);
+  return static_cast<size_t>(B) * Hq * per_bh;
+}
+
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? HD_OK : HD_ERR_CUDA; }
 
 }  // namespace
@@ -158,7 +169,7 @@ size_t hd_attn_bwd_workspace_bytes(int B, int L, int n, int Hq, int Hkv, int D,
   const size_t Sq = final_stream_queries_only ? static_cast<size_t>(L)
                                               : static_cast<size_t>(n) * static_cast<size_t>(L);
   const size_t rows = static_cast<size_t>(B) * Sq * static_cast<size_t>(Hq);
-  return align256(rows * static_cast<size_t>(D) * 4) + align256(rows * 4);
+  return align256(rows * static_cast<size_t>(D) * 4) + 2 * align256(packed_rows(B, L, n, Hq, final_stream_queries_only) * 4);
 }
 
 int hd_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
@@ -183,7 +194,10 @@ int hd_attn_bwd(const void* q, const void* k, const void* v, const void* out, co
   p.dv = static_cast<__nv_bfloat16*>(dv);
   const size_t rows = static_cast<size_t>(B) * p.Sq * Hq;
   p.dq_acc = static_cast<float*>(workspace);
-  p.delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(rows * D * 4));
+  const size_t npk = packed_rows(B, L, n, Hq, final_stream_queries_only);
+  p.lse2p = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(rows * D * 4));
+  p.deltap = reinterpret_cast<float*>(reinterpret_cast<char*>(p.lse2p) + align256(npk * 4));
+  p.lq_pad = static_cast<int>(pad64(p.Lq));
   return from_cuda(launch_attn_bwd(p, static_cast<cudaStream_t>(stream)));
 }
 

@@ -8,7 +8,8 @@
 //   dQ = scale dS K,  dK = scale sum_group dS^T Q,  dV = sum_group P^T dO.
 //
 // Kernels on the caller's stream:
-//   1. bwd_pre:   D = rowsum(dO * O) (fp32, LSE layout); zero the fp32 dQ
+//   1. bwd_pre:   D = rowsum(dO * O) and LSE * log2(e), both packed per
+//                 problem (row-contiguous, padded to 64 rows); zero the fp32 dQ
 //                 accumulator.
 //   2. attn_bwd_tc_kernel (attn_bwd_tc.cu): dK, dV and the fp32 dQ sums.
 //   3. bwd_zero_unread_kv (INTRA with final-stream-only queries only): the dK /
@@ -40,7 +41,21 @@ __global__ void bwd_pre_kernel(const AttnParams p) {
   }
 #pragma unroll
   for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-  if (lane == 0) p.delta[(b * p.Hq + h) * p.Sq + i] = acc;
+  // packed row statistics of problem (b, h, grp), row r
+  const bool intra_groups = p.mode == HD_INTRA && !p.final_only;
+  const long long grp = intra_groups ? i % p.n : 0;
+  const long long r = intra_groups ? i / p.n : i;
+  const long long pk = ((b * p.Hq + h) * p.groups + grp) * p.lq_pad;
+  if (lane == 0) {
+    p.deltap[pk + r] = acc;
+    p.lse2p[pk + r] = p.lse[(b * p.Hq + h) * p.Sq + i] * 1.4426950408889634074f;
+  }
+  if (r == p.Lq - 1) {  // zero the padding rows after the problem's last row
+    for (int j = lane; j < p.lq_pad - p.Lq; j += 32) {
+      p.deltap[pk + p.Lq + j] = 0.f;
+      p.lse2p[pk + p.Lq + j] = 0.f;
+    }
+  }
   float4* z = reinterpret_cast<float4*>(p.dq_acc + row * p.D);
   for (int c = lane; c < p.D / 4; c += 32) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
 }

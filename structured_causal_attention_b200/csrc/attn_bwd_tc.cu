@@ -14,8 +14,8 @@
 //   dK  += dS^T Q     (M 128 keys, N D)            } the whole group
 //   dQ^T = K^T dS^T   (M D, N 64 queries)           into the S^T buffer
 // Roles (12 warps):
-//   warp 0      TMA: K, V once; Q and dO tiles (2 stages); its lanes also stage
-//               the tile's LSE and D values in shared memory.
+//   warp 0      TMA: K, V once; Q and dO tiles (2 stages) plus the tile's
+//               packed LSE and D rows (bulk copies).
 //   warp 1      TMEM allocation; lane 0 issues the MMAs.
 //   warps 4-7   one key row per thread: P^T = exp2(S^T - LSE), dS^T = P^T (dP^T - D),
 //               written as bf16 into shared memory in the MMA operand layout;
@@ -37,7 +37,6 @@ constexpr int kKN = 128;   // keys per CTA
 constexpr int kQM = 64;    // query rows per iteration
 constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
-constexpr float kLog2e = 1.4426950408889634074f;
 
 template <int D>
 struct BtSmem {
@@ -65,7 +64,7 @@ struct BtSmem {
 // barrier indices
 enum {
   B_KV = 0,   // K and V loaded
-  B_QF = 1,   // [2] Q/dO (+ LSE, D) of a stage loaded: 1 tx arrival + 32 lane arrivals
+  B_QF = 1,   // [2] Q, dO and the packed LSE / D rows of a stage loaded
   B_QE = 3,   // [2] stage free (MMA commit)
   B_SF = 5,   // [2] S^T / dP^T ready (MMA commit)
   B_PF = 7,   // P^T / dS^T written (4 warp arrivals)
@@ -112,17 +111,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int c_last = min(c0 + kKN, p.Lk) - 1;
   const int rmin = (c0 - p.bb <= 0) ? 0 : (c0 - p.bb + p.a - 1) / p.a;
   const int rmax = min(p.Lq - 1, (c_last + p.win - 1 - p.bb) / p.a);
-  const int qt_lo = rmin / kQM;
-  const int nqt = rmin <= rmax ? rmax / kQM - qt_lo + 1 : 0;
+  const int qt_lo = rmin / kQM, qt_hi = rmax / kQM;
+  const int nqt = rmin <= rmax ? qt_hi - qt_lo + 1 : 0;
   const int total = g * nqt;
-  auto iter_head = [&](int it) { return hk * g + it / nqt; };
-  auto iter_row0 = [&](int it) { return (qt_lo + it % nqt) * kQM; };
+  // Query tiles from the last one down, the group's heads inner: the CTAs of
+  // one (batch, KV head) then walk the same tiles at the same time, so Q, dO
+  // and the dQ accumulator tiles they share stay in L2.
+  auto iter_head = [&](int it) { return hk * g + it % g; };
+  auto iter_row0 = [&](int it) { return (qt_hi - it / g) * kQM; };
   auto jq_of = [&](int h) { return (intra && !p.final_only) ? grp * p.Hq + h : h; };
 
   if (tid == 0) {
     for (int i = 0; i < SM::NBAR; ++i) {
       uint32_t cnt = 1;
-      if (i == B_QF || i == B_QF + 1) cnt = 33;
       if (i == B_PF || i == B_DE || i == B_DE + 1) cnt = 4;
       tc::mbar_init(bar(i), cnt);
     }
@@ -153,33 +154,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tma_load_4d(sV + s * SM::KSUB, &tmV, bar(B_KV), s * 64, jk, c0, b);
       }
     }
-    for (int it = 0; it < total; ++it) {
+    for (int it = 0; lane == 0 && it < total; ++it) {
       const int st = it & 1;
       if (!tc::mbar_wait(bar(B_QE + st), ((it >> 1) & 1) ^ 1, abort_flag, p.status)) break;
       const int h = iter_head(it), rq0 = iter_row0(it), jq = jq_of(h);
       if (lane == 0) {
-        tc::mbar_expect_tx(bar(B_QF + st), 2 * NSUB * SM::QSUB);
+        const long long pk = ((static_cast<long long>(b) * p.Hq + h) * p.groups + grp) * p.lq_pad + rq0;
+        tc::mbar_expect_tx(bar(B_QF + st), 2 * NSUB * SM::QSUB + 2 * kQM * 4);
 #pragma unroll
         for (int s = 0; s < NSUB; ++s) {
           tc::tma_load_4d(sQ + (st * NSUB + s) * SM::QSUB, &tmQ, bar(B_QF + st), s * 64, jq, rq0, b);
           tc::tma_load_4d(sDO + (st * NSUB + s) * SM::QSUB, &tmDO, bar(B_QF + st), s * 64, jq, rq0, b);
         }
+        tc::bulk_load(sbase + SM::L_OFF + st * kQM * 4, p.lse2p + pk, kQM * 4, bar(B_QF + st));
+        tc::bulk_load(sbase + SM::DL_OFF + st * kQM * 4, p.deltap + pk, kQM * 4, bar(B_QF + st));
       }
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const int rr = lane + 32 * k, r = rq0 + rr;
-        float l2 = 0.f, dl = 0.f;
-        if (r < p.Lq) {
-          const long long li = (static_cast<long long>(b) * p.Hq + h) * p.Sq +
-                               static_cast<long long>(grp) * p.qs_step +
-                               static_cast<long long>(r) * p.q_rstride;
-          l2 = p.lse[li] * kLog2e;
-          dl = p.delta[li];
-        }
-        sL[st * kQM + rr] = l2;
-        sDl[st * kQM + rr] = dl;
-      }
-      tc::mbar_arrive(bar(B_QF + st));
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
@@ -258,42 +247,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool full = (c0 + kKN - 1 <= p.a * rq0 + p.bb) &&
                         (c0 > p.a * (rq0 + kQM - 1) + p.bb - p.win) && (c0 + kKN <= p.Lk) &&
                         (rq0 + kQM <= p.Lq);
-      if (it > 0) {
-        if (!tc::mbar_wait(bar(B_PE), (it - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-      }
+      uint32_t pp[32], dd[32];  // bf16 pairs of P^T and dS^T for the 64 queries
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t sr[32], dr[32];
         tc::tmem_ld32(tmem + tq + 128 * x + half * 32, sr);
         tc::tmem_ld32(tmem + tq + 128 * x + 64 + half * 32, dr);
         tc::tmem_wait_ld();
-        float pv[32], ds[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int rl = half * 32 + j;
-          const float l2 = sL[st * kQM + rl];
-          float pj = fast_exp2(fmaf(__uint_as_float(sr[j]), p.scale_log2, -l2));
-          if (!full) {
-            const int r = rq0 + rl;
-            const int hi = p.a * r + p.bb;
-            if (!(r < p.Lq && c <= hi && c > hi - p.win && c < p.Lk)) pj = 0.f;
+        for (int j = 0; j < 32; j += 2) {
+          float pj[2], dj[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int rl = half * 32 + j + e;
+            float pv = fast_exp2(fmaf(__uint_as_float(sr[j + e]), p.scale_log2, -sL[st * kQM + rl]));
+            if (!full) {
+              const int r = rq0 + rl;
+              const int hi = p.a * r + p.bb;
+              if (!(r < p.Lq && c <= hi && c > hi - p.win && c < p.Lk)) pv = 0.f;
+            }
+            pj[e] = pv;
+            dj[e] = pv * (__uint_as_float(dr[j + e]) - sDl[st * kQM + rl]);
           }
-          pv[j] = pj;
-          ds[j] = pj * (__uint_as_float(dr[j]) - sDl[st * kQM + rl]);
+          pp[half * 16 + j / 2] = pack_bf16(pj[0], pj[1]);
+          dd[half * 16 + j / 2] = pack_bf16(dj[0], dj[1]);
         }
+      }
+      // the MMAs of the previous tile have finished reading P^T / dS^T
+      if (it > 0) {
+        if (!tc::mbar_wait(bar(B_PE), (it - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+      }
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int ch = half * 4 + k;
-          const uint32_t off = row * 128 + ((ch ^ (row & 7)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(sP + off),
-                       "r"(pack_bf16(pv[8 * k], pv[8 * k + 1])), "r"(pack_bf16(pv[8 * k + 2], pv[8 * k + 3])),
-                       "r"(pack_bf16(pv[8 * k + 4], pv[8 * k + 5])), "r"(pack_bf16(pv[8 * k + 6], pv[8 * k + 7]))
-                       : "memory");
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(sDS + off),
-                       "r"(pack_bf16(ds[8 * k], ds[8 * k + 1])), "r"(pack_bf16(ds[8 * k + 2], ds[8 * k + 3])),
-                       "r"(pack_bf16(ds[8 * k + 4], ds[8 * k + 5])), "r"(pack_bf16(ds[8 * k + 6], ds[8 * k + 7]))
-                       : "memory");
-        }
+      for (int ch = 0; ch < 8; ++ch) {
+        const uint32_t off = row * 128 + ((ch ^ (row & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(sP + off), "r"(pp[4 * ch]),
+                     "r"(pp[4 * ch + 1]), "r"(pp[4 * ch + 2]), "r"(pp[4 * ch + 3])
+                     : "memory");
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(sDS + off), "r"(dd[4 * ch]),
+                     "r"(dd[4 * ch + 1]), "r"(dd[4 * ch + 2]), "r"(dd[4 * ch + 3])
+                     : "memory");
       }
       tc::fence_async_smem();
       tc::tc_fence_before();

@@ -40,7 +40,9 @@ struct AttnParams {
   // backward only
   const __nv_bfloat16* dout;
   float* dq_acc;        // fp32 accumulator, q's layout
-  float* delta;         // fp32 rowsum(dO * O), lse's layout
+  float* lse2p;         // LSE * log2(e), packed per problem: [B][Hq][groups][lq_pad]
+  float* deltap;        // rowsum(dO * O), same packed layout
+  int lq_pad;           // Lq rounded up to 64 (padding rows hold zeros)
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;

@@ -68,8 +68,9 @@ def test_fwd_rejects(lib, kw, code):
 def test_bwd_workspace_and_rejects(lib):
     ws = hd.hd_attn_bwd_workspace_bytes(2, 16, 4, 8, 2, 128, 0)
     rows = 2 * 64 * 8
-    assert ws == rows * 128 * 4 + rows * 4
-    assert hd.hd_attn_bwd_workspace_bytes(2, 16, 4, 8, 2, 128, 1) == 2 * 16 * 8 * (128 * 4 + 4)
+    # fp32 dQ accumulator + LSE and D rows packed per problem, padded to 64 rows
+    assert ws == rows * 128 * 4 + 2 * (2 * 8 * 4 * 64 * 4)
+    assert hd.hd_attn_bwd_workspace_bytes(2, 16, 4, 8, 2, 128, 1) == 2 * 16 * 8 * 128 * 4 + 2 * (2 * 8 * 64 * 4)
     assert hd.hd_attn_bwd_workspace_bytes(0, 16, 4, 8, 2, 128, 0) == 0
     L = hd.lib()
     args = [FAKE] * 9 + [2, 16, 4, 8, 2, 128, hd.INTRA, 1, 0, 0.1]

@@ -13,15 +13,15 @@
 //   dV  += P^T dO     (M 128 keys, N D)            } accumulated in TMEM across
 //   dK  += dS^T Q     (M 128 keys, N D)            } the whole group
 //   dQ^T = K^T dS^T   (M D, N 64 queries)           into the S^T buffer
-// Roles (12 warps):
-//   warp 0      TMA: K, V once; Q and dO tiles (2 stages) plus the tile's
-//               packed LSE and D rows (bulk copies).
-//   warp 1      TMEM allocation; lane 0 issues the MMAs.
-//   warps 4-7   one key row per thread: P^T = exp2(S^T - LSE), dS^T = P^T (dP^T - D),
+// Roles (10 warps):
+//   warps 0-3   one key row per thread: P^T = exp2(S^T - LSE), dS^T = P^T (dP^T - D),
 //               written as bf16 into shared memory in the MMA operand layout;
 //               at the end dK (scaled) and dV go out through TMA stores.
-//   warps 8-11  one head-dim row per thread: dQ^T from TMEM into an fp32 tile,
+//   warps 4-7   one head-dim row per thread: dQ^T from TMEM into an fp32 tile,
 //               added into the fp32 dQ accumulator with a TMA bulk reduce-add.
+//   warp 8      TMA: K, V once; Q and dO tiles (2 stages) plus the tile's
+//               packed LSE and D rows (bulk copies).
+//   warp 9      TMEM allocation; lane 0 issues the MMAs.
 // Every mbarrier wait is bounded (HD_ERR_TIMEOUT, then every role leaves).
 #include <cuda.h>
 
@@ -35,7 +35,7 @@ namespace {
 
 constexpr int kKN = 128;   // keys per CTA
 constexpr int kQM = 64;    // query rows per iteration
-constexpr int kThreads = 384;
+constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 
 template <int D>
@@ -96,9 +96,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (p.status && *reinterpret_cast<volatile int*>(p.status) == HD_ERR_TIMEOUT) return;
 
-  // ---- problem of this CTA: key tile kt of (b, hk, grp)
+  // ---- problem of this CTA: key tile kt of (b, hk, grp); key-tile-major grid,
+  // low key tiles (which see the most queries) first
   const int bkg = p.B * p.Hkv * p.groups;
-  const int kt = static_cast<int>(blockIdx.x / bkg);  // low key tiles see the most queries
+  const int kt = static_cast<int>(blockIdx.x / bkg);
   int y = static_cast<int>(blockIdx.x % bkg);
   const int grp = y % p.groups;
   y /= p.groups;
@@ -130,7 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == 9) {
     tc::tmem_alloc(sbase + SM::SLOT_OFF, kTmemCols);
     tc::tmem_relinquish();
   }
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // dK at 256, dV at 256 + D.
   const uint32_t tdK = tmem + 256, tdV = tmem + 256 + D;
 
-  if (warp == 0) {
+  if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tc::tma_prefetch_desc(&tmQ);
@@ -170,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::bulk_load(sbase + SM::DL_OFF + st * kQM * 4, p.deltap + pk, kQM * 4, bar(B_QF + st));
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0 && total > 0) {
       constexpr uint32_t idSP = tc::idesc_bf16_f32(128, kQM, 0, 0);  // S^T, dP^T
@@ -233,11 +234,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc::mma_commit(bar(B_END));
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp < 4) {
     // ------------------------------------------------ P^T, dS^T (one key per thread)
-    const int row = tid - 128;
+    const int row = tid;
     const int c = c0 + row;
-    const uint32_t tq = static_cast<uint32_t>((warp - 4) * 32) << 16;
+    const uint32_t tq = static_cast<uint32_t>(warp * 32) << 16;
     bool ok = true;
     for (int it = 0; it < total; ++it) {
       const int x = it & 1, st = it & 1;
@@ -334,10 +335,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc::tma_store_commit_and_wait();
     }
-  } else if (warp >= 8) {
+  } else {
     // ------------------------------------- dQ^T readout (one head-dim row per thread)
-    const int d = tid - 256;
-    const uint32_t tq = static_cast<uint32_t>((warp - 8) * 32) << 16;
+    const int d = tid - 128;
+    const uint32_t tq = static_cast<uint32_t>((warp - 4) * 32) << 16;
     for (int it = 0; it < total; ++it) {
       const int x = it & 1;
       if (!tc::mbar_wait(bar(B_DF + x), (it >> 1) & 1, abort_flag, p.status)) break;
@@ -377,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 9) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, kTmemCols);
   }

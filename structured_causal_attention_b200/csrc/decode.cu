@@ -121,6 +121,14 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
     srow[hr] = rvalid[hr] ? row / g : 0;
     prow[hr] = T * p.n + srow[hr];
   }
+  // INTRA: key c is visible iff c % n == s. Blocks start at multiples of 64,
+  // so c % n = (block base % n + offset % n) mod n: the offsets' residues are
+  // fixed per thread, the base's residue is one modulo per block.
+  int om[2][2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) om[j][e] = (warp * 16 + j * 8 + (lane & 3) * 2 + e) % p.n;
   float o[NDT][4];
 #pragma unroll
   for (int j = 0; j < NDT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
@@ -145,6 +153,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
       mma_bf16_16816(s[1], qf[kk], b2, b3);
     }
     const int cbase = cs + bi * kDecBlk + warp * 16;
+    const int bres = (p.mode == HD_INTRA) ? (cs + bi * kDecBlk) % p.n : 0;
 #pragma unroll
     for (int j = 0; j < 2; ++j)
 #pragma unroll
@@ -152,7 +161,11 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
         const int hr = e >> 1;
         const int c = cbase + j * 8 + (lane & 3) * 2 + (e & 1);
         bool vis = rvalid[hr] && c < ce && c <= prow[hr];
-        if (p.mode == HD_INTRA) vis = vis && (c % p.n == srow[hr]);
+        if (p.mode == HD_INTRA) {
+          int res = bres + om[j][e & 1];
+          res -= (res >= p.n) ? p.n : 0;
+          vis = vis && (res == srow[hr]);
+        }
         if (p.mode == HD_CROSS_WINDOW) vis = vis && (prow[hr] - c < p.win);
         if (!vis) s[j][e] = -INFINITY;
       }
@@ -314,7 +327,9 @@ void decode_split_plan(int B, int n, int Tcap, int Hq, int Hkv, int* mt, int* sp
   const long long keys = static_cast<long long>(Tcap) * n;
   const long long target = 148LL * 2 * 4;  // 4 waves of 2 resident CTAs per SM
   long long sp = (target + units - 1) / units;
-  const long long max_sp = (keys + kDecBlk - 1) / kDecBlk;
+  // at least 8 blocks (512 keys) per split, so that short caches are not cut
+  // into many tiny chunks that the combine step then has to walk
+  const long long max_sp = (keys + 8 * kDecBlk - 1) / (8 * kDecBlk);
   if (sp > max_sp) sp = max_sp;
   if (sp < 1) sp = 1;
   long long ch = (keys + sp - 1) / sp;

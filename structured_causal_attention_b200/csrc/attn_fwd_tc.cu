@@ -8,23 +8,28 @@
 // section "隐式序列缩放的技术细节" step 2 (causal attention over the expanded
 // sequence).
 //
-// One CTA = one 128-row query tile of one (batch, head, stream group).
-//   warp 0      TMA producer: Q once, then K and V tiles of 128 keys into a
-//               2-stage ring (128-byte swizzle). The 4-D tensor maps are
+// One CTA = two consecutive 128-row query tiles of one (batch, head, stream
+// group); they share every K/V tile the CTA loads.
+//   warps 0-3 / 4-7  softmax warpgroup of query tile 0 / 1, one row per thread
+//               (= TMEM lane): tcgen05.ld of the S row, mask on boundary tiles,
+//               online softmax in base 2, P as bf16 pairs written back into the
+//               upper S columns of TMEM (tcgen05.st). The running max is only raised
+//               when a tile's max exceeds it by more than 2^8, so the O
+//               accumulator is rescaled in TMEM rarely; the final 1/l and LSE
+//               make the result exact either way.
+//   warp 8      TMA producer: both Q tiles once, then K and V tiles of 128 keys
+//               into a 2-stage ring (128-byte swizzle). The 4-D tensor maps are
 //               (d, head-or-stream*head, row, batch), so an INTRA stream is read
 //               as a contiguous causal problem (row stride n*H*D), with no copy.
-//   warp 1      allocates TMEM; lane 0 issues every tcgen05.mma:
-//               S_i = Q K_i^T into one of two TMEM S buffers (M=128, N=128),
-//               O += P_i V_i into the TMEM O accumulator (M=128, N=D, V read
-//               MN-major straight from its TMA tile).
-//   warps 4-7   softmax warpgroup, one query row per thread (= TMEM lane):
-//               tcgen05.ld of the S row, mask on boundary tiles, online softmax
-//               in base 2, P (bf16) into shared memory in the MMA's K-major
-//               128-byte-swizzled layout. The running max is only raised when
-//               a tile's max exceeds it by more than 2^8, so the O accumulator
-//               is rescaled in TMEM rarely; the final 1/l and LSE make the
-//               result exact either way.
-// S_{i+1} runs on the tensor core while the softmax of tile i runs.
+//   warp 9      allocates TMEM (2 x [S/P 128 columns | O D columns]); lane 0
+//               issues every tcgen05.mma in the order
+//                   PV_0(j), S_0(j+1), PV_1(j), S_1(j+1)
+//               so one tile's MMAs run while the other tile's softmax works.
+//               S = Q K^T (M=128, N=128, both operands from shared memory);
+//               O += P V (M=128, N=D, P from TMEM, V MN-major from its TMA tile).
+// MMAs from one thread execute in order, so when S_q(j) is complete, PV_q(j-1)
+// (issued before it) has finished reading P and updating O: the softmax may
+// then rescale O and overwrite P without another wait.
 // Every mbarrier wait is bounded; on expiry the kernel records HD_ERR_TIMEOUT,
 // every role leaves its loop, TMEM is freed and the kernel returns.
 #include <cuda.h>
@@ -37,33 +42,32 @@ namespace hd {
 
 namespace {
 
-constexpr int kBM = 128;  // query rows per CTA
-constexpr int kBN = 128;  // keys per tile
-constexpr int kThreads = 256;
+constexpr int kBM = 128;  // query rows per tile (2 tiles per CTA)
+constexpr int kBN = 128;  // keys per K/V tile
+constexpr int kThreads = 320;
 constexpr int kSub = 128 * 128;  // bytes of one [128 rows][64 bf16] swizzled sub-tile
 constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleLog2 = 8.f;  // raise the running max only past 2^8
 
 template <int D>
 struct TcSmem {
   static constexpr int NSUB = D / 64;
   static constexpr int Q_BYTES = kBM * D * 2;
   static constexpr int KV_BYTES = kBN * D * 2;
-  static constexpr int P_BYTES = kBM * kBN * 2;
-  static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = Q_OFF + Q_BYTES;
-  static constexpr int V_OFF = K_OFF + 2 * KV_BYTES;
-  static constexpr int P_OFF = V_OFF + 2 * KV_BYTES;
-  static constexpr int BAR_OFF = P_OFF + P_BYTES;
-  // barriers: q_full, k_full[2], v_full[2], kv_empty[2], s_full[2], s_free[2], p_full, o_done
+  static constexpr int Q_OFF = 0;                          // 2 query tiles
+  static constexpr int K_OFF = Q_OFF + 2 * Q_BYTES;        // 2 stages
+  static constexpr int V_OFF = K_OFF + 2 * KV_BYTES;       // 2 stages
+  static constexpr int BAR_OFF = V_OFF + 2 * KV_BYTES;
+  // q_full, k_full[2], v_full[2], kv_empty[2], s_full[2], p_full[2], o_final[2]
   static constexpr int NBAR = 13;
-  static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;  // TMEM base address
+  static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;
   static constexpr int ABORT_OFF = SLOT_OFF + 4;
-  // + alignment slack; at least 120 KB so that one CTA (and one 512-column
-  // TMEM allocation) is resident per SM
-  static constexpr int TOTAL = (ABORT_OFF + 4 + 1024) > 120 * 1024 ? (ABORT_OFF + 4 + 1024) : 120 * 1024;
+  static constexpr int USED = ABORT_OFF + 4 + 1024;
+  // at least 120 KB so that one CTA (one 512-column TMEM allocation) is resident per SM
+  static constexpr int TOTAL = USED > 120 * 1024 ? USED : 120 * 1024;
 };
 
-enum { B_QF = 0, B_KF = 1, B_VF = 3, B_KE = 5, B_SF = 7, B_SE = 9, B_PF = 11, B_OD = 12 };
+enum { B_QF = 0, B_KF = 1, B_VF = 3, B_KE = 5, B_SF = 7, B_PF = 9, B_OF = 11 };
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -75,21 +79,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
-  const uint32_t sQ = sbase + SM::Q_OFF, sK = sbase + SM::K_OFF, sV = sbase + SM::V_OFF,
-                 sP = sbase + SM::P_OFF;
+  const uint32_t sQ = sbase + SM::Q_OFF, sK = sbase + SM::K_OFF, sV = sbase + SM::V_OFF;
   auto bar = [&](int i) { return sbase + SM::BAR_OFF + 8u * i; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + SM::ABORT_OFF);
-  const uint32_t slot = sbase + SM::SLOT_OFF;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // A timeout recorded by an earlier CTA (or call) is sticky until the status
   // word is cleared: skip the work instead of waiting again.
   if (p.status && *reinterpret_cast<volatile int*>(p.status) == HD_ERR_TIMEOUT) return;
 
-  // ---- problem of this CTA
+  // ---- problem of this CTA: query tiles 2*pq and 2*pq+1
   const int bhg = p.B * p.Hq * p.groups;
   const int num_qt = (p.Lq + kBM - 1) / kBM;
-  const int qt = num_qt - 1 - static_cast<int>(blockIdx.x / bhg);  // heavy tiles first
+  const int num_pairs = (num_qt + 1) / 2;
+  const int pq = num_pairs - 1 - static_cast<int>(blockIdx.x / bhg);  // heavy pairs first
   int y = static_cast<int>(blockIdx.x % bhg);
   const int grp = y % p.groups;
   y /= p.groups;
@@ -99,40 +102,55 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool intra = p.mode == HD_INTRA;
   const int jq = (intra && !p.final_only) ? grp * p.Hq + h : h;
   const int jk = intra ? (p.final_only ? p.n - 1 : grp) * p.Hkv + hk : hk;
-  const int r0 = qt * kBM;
-  const int r_last = min(r0 + kBM, p.Lq) - 1;
-  const int kmax = min(p.Lk - 1, p.a * r_last + p.bb);
-  const int kmin = max(0, p.a * r0 + p.bb - p.win + 1);
-  const int kt_lo = kmin / kBN;
-  const int nt = kmax / kBN - kt_lo + 1;
+  const int r0 = 2 * pq * kBM;
+  // K/V tile range [lo_q, hi_q] of each query tile (empty when the tile has no rows)
+  int lo[2], hi[2];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const int rq = r0 + q * kBM;
+    if (rq >= p.Lq) {
+      lo[q] = 1;
+      hi[q] = 0;
+      continue;
+    }
+    const int rl = min(rq + kBM, p.Lq) - 1;
+    lo[q] = max(0, p.a * rq + p.bb - p.win + 1) / kBN;
+    hi[q] = min(p.Lk - 1, p.a * rl + p.bb) / kBN;
+  }
+  const int kt_lo = lo[1] <= hi[1] ? min(lo[0], lo[1]) : lo[0];
+  const int kt_hi = max(hi[0], hi[1]);
+  const int nkv = kt_hi - kt_lo + 1;
+  auto in_range = [&](int q, int j) { return j >= lo[q] && j <= hi[q]; };
 
   if (tid == 0) {
     // softmax warps arrive once per warp (4); everything else arrives once
-    for (int i = 0; i < SM::NBAR; ++i)
-      tc::mbar_init(bar(i), (i == B_SE || i == B_SE + 1 || i == B_PF) ? 4 : 1);
+    for (int i = 0; i < SM::NBAR; ++i) tc::mbar_init(bar(i), (i == B_PF || i == B_PF + 1) ? 4 : 1);
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
-  if (warp == 1) {
-    tc::tmem_alloc(slot, kTmemCols);
+  if (warp == 9) {
+    tc::tmem_alloc(sbase + SM::SLOT_OFF, kTmemCols);
     tc::tmem_relinquish();
   }
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sgen + SM::SLOT_OFF);
-  const uint32_t tS = tmem, tO = tmem + 256;  // S buffers at columns 0 and 128, O at 256
+  // tile q: S at 256q (P, as bf16 pairs, in its columns 64..127), O at 256q + 128
 
-  if (warp == 0) {
+  if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tc::tma_prefetch_desc(&tmQ);
       tc::tma_prefetch_desc(&tmK);
       tc::tma_prefetch_desc(&tmV);
-      tc::mbar_expect_tx(bar(B_QF), SM::Q_BYTES);
+      tc::mbar_expect_tx(bar(B_QF), 2 * SM::Q_BYTES);
 #pragma unroll
-      for (int s = 0; s < NSUB; ++s) tc::tma_load_4d(sQ + s * kSub, &tmQ, bar(B_QF), s * 64, jq, r0, b);
-      for (int i = 0; i < nt; ++i) {
+      for (int q = 0; q < 2; ++q)
+#pragma unroll
+        for (int s = 0; s < NSUB; ++s)
+          tc::tma_load_4d(sQ + q * SM::Q_BYTES + s * kSub, &tmQ, bar(B_QF), s * 64, jq, r0 + q * kBM, b);
+      for (int i = 0; i < nkv; ++i) {
         const int st = i & 1;
         if (!tc::mbar_wait(bar(B_KE + st), ((i >> 1) & 1) ^ 1, abort_flag, p.status)) break;
         const int c0 = (kt_lo + i) * kBN;
@@ -146,146 +164,177 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::tma_load_4d(sV + st * SM::KV_BYTES + s * kSub, &tmV, bar(B_VF + st), s * 64, jk, c0, b);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = tc::idesc_bf16_f32(kBM, kBN, 0, 0);
       constexpr uint32_t idO = tc::idesc_bf16_f32(kBM, D, 0, 1);
-      auto issue_S = [&](int buf, int st) {
+      auto issue_S = [&](int q, int st) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
-          tc::mma_ss(tS + buf * 128, tc::smem_desc_sw128(sQ + off, 16, 1024),
+          tc::mma_ss(tmem + 256 * q, tc::smem_desc_sw128(sQ + q * SM::Q_BYTES + off, 16, 1024),
                      tc::smem_desc_sw128(sK + st * SM::KV_BYTES + off, 16, 1024), idS, kk > 0);
         }
+        tc::mma_commit(bar(B_SF + q));
       };
+      int pf_count[2] = {0, 0};
       bool ok = tc::mbar_wait(bar(B_QF), 0, abort_flag, p.status) &&
                 tc::mbar_wait(bar(B_KF), 0, abort_flag, p.status);
       if (ok) {
         tc::tc_fence_after();
-        issue_S(0, 0);
-        tc::mma_commit(bar(B_SF));
-      }
-      for (int i = 0; ok && i < nt; ++i) {
-        const int st = i & 1;
-        if (i + 1 < nt) {
-          const int s1 = (i + 1) & 1;
-          ok = tc::mbar_wait(bar(B_KF + s1), ((i + 1) >> 1) & 1, abort_flag, p.status);
-          if (ok && i + 1 >= 2)
-            ok = tc::mbar_wait(bar(B_SE + s1), (((i + 1) >> 1) - 1) & 1, abort_flag, p.status);
-          if (!ok) break;
-          tc::tc_fence_after();
-          issue_S(s1, s1);
-          tc::mma_commit(bar(B_SF + s1));
-        }
-        ok = tc::mbar_wait(bar(B_PF), i & 1, abort_flag, p.status) &&
-             tc::mbar_wait(bar(B_VF + st), (i >> 1) & 1, abort_flag, p.status);
-        if (!ok) break;
-        tc::tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t ad = tc::smem_desc_sw128(sP + (kk >> 2) * kSub + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = tc::smem_desc_sw128(sV + st * SM::KV_BYTES + kk * 2048, kSub, 1024);
-          tc::mma_ss(tO, ad, bd, idO, (i > 0 || kk > 0) ? 1u : 0u);
+        for (int q = 0; q < 2; ++q)
+          if (in_range(q, kt_lo)) issue_S(q, 0);
+      }
+      for (int i = 0; ok && i < nkv; ++i) {
+        const int j = kt_lo + i, st = i & 1, s1 = (i + 1) & 1;
+        bool v_ready = false, k_next_ready = false;
+#pragma unroll
+        for (int q = 0; q < 2 && ok; ++q) {
+          if (in_range(q, j)) {
+            ok = tc::mbar_wait(bar(B_PF + q), pf_count[q] & 1, abort_flag, p.status);
+            if (ok && !v_ready) ok = tc::mbar_wait(bar(B_VF + st), (i >> 1) & 1, abort_flag, p.status);
+            if (!ok) break;
+            v_ready = true;
+            ++pf_count[q];
+            tc::tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < kBN / 16; ++kk)
+              tc::mma_ts(tmem + 256 * q + 128, tmem + 256 * q + 64 + kk * 8,
+                         tc::smem_desc_sw128(sV + st * SM::KV_BYTES + kk * 2048, kSub, 1024), idO,
+                         (j > lo[q] || kk > 0) ? 1u : 0u);
+            if (j == hi[q]) tc::mma_commit(bar(B_OF + q));
+          }
+          if (in_range(q, j + 1)) {
+            if (!k_next_ready) {
+              ok = tc::mbar_wait(bar(B_KF + s1), ((i + 1) >> 1) & 1, abort_flag, p.status);
+              if (!ok) break;
+              k_next_ready = true;
+              tc::tc_fence_after();
+            }
+            issue_S(q, s1);
+          }
         }
-        tc::mma_commit(bar(B_OD));
         tc::mma_commit(bar(B_KE + st));
       }
     }
-  } else if (warp >= 4) {
-    // --------------------------------------------------------- softmax warpgroup
-    const int row = tid - 128;
-    const int r = r0 + row;
-    const uint32_t tq = static_cast<uint32_t>((warp - 4) * 32) << 16;
-    const int hi = p.a * r + p.bb;
-    const int lo = hi - p.win;
+  } else {
+    // ------------------------------------------------------ softmax warpgroups
+    const int q = warp >> 2;  // query tile of this warpgroup
+    const int row = tid & 127;
+    const int r = r0 + q * kBM + row;
+    const uint32_t tq = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + 256 * q + tq, tO = tS + 128;
+    const int rq0 = r0 + q * kBM;
+    const int rq_last = min(rq0 + kBM, p.Lq) - 1;
+    const int hi_r = p.a * r + p.bb;
+    const int lo_r = hi_r - p.win;
+    const int my_lo = q ? lo[1] : lo[0], my_hi = q ? hi[1] : hi[0];
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int i = 0; i < nt; ++i) {
-      const int st = i & 1;
-      if (!tc::mbar_wait(bar(B_SF + st), (i >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+    int t = 0;
+    for (int j = my_lo; j <= my_hi; ++j, ++t) {
+      if (!tc::mbar_wait(bar(B_SF + q), t & 1, abort_flag, p.status)) { ok = false; break; }
       tc::tc_fence_after();
-      uint32_t sr[kBN];
+      const int c0 = j * kBN;
+      const bool full = (c0 + kBN - 1 <= p.a * rq0 + p.bb) &&
+                        (c0 > p.a * rq_last + p.bb - p.win) && (c0 + kBN <= p.Lk);
+      // Three TMEM round trips per tile with at most 64 scores live: keys 0-63
+      // (max), keys 64-127 (max, then their P), keys 0-63 again (their P).
+      // P goes to columns 64..127 as bf16 pairs (keys 0-63 -> 64..95,
+      // keys 64-127 -> 96..127), i.e. only over scores already read.
+      auto mask_half = [&](uint32_t* v, int half) {
+        if (!full) {
 #pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) tc::tmem_ld32(tS + tq + st * 128 + c * 32, sr + c * 32);
-      tc::tmem_wait_ld();
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(bar(B_SE + st));
-      float* s = reinterpret_cast<float*>(sr);
-      const int c0 = (kt_lo + i) * kBN;
-      const bool full = (c0 + kBN - 1 <= p.a * r0 + p.bb) &&
-                        (c0 > p.a * r_last + p.bb - p.win) && (c0 + kBN <= p.Lk);
-      if (!full) {
-#pragma unroll
-        for (int j = 0; j < kBN; ++j) {
-          const int c = c0 + j;
-          if (!(c <= hi && c > lo && c < p.Lk)) s[j] = -INFINITY;
+          for (int e = 0; e < 64; ++e) {
+            const int key = c0 + half * 64 + e;
+            if (!(key <= hi_r && key > lo_r && key < p.Lk)) v[e] = __float_as_uint(-INFINITY);
+          }
         }
-      }
-      float mx = -INFINITY;
+      };
+      auto exp_half = [&](const uint32_t* v, int half, float m_use) {
 #pragma unroll
-      for (int j = 0; j < kBN; ++j) mx = fmaxf(mx, s[j]);
-      const float m_tile = mx * p.scale_log2;
-      if (i > 0) {
-        if (!tc::mbar_wait(bar(B_OD), (i - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-        tc::tc_fence_after();
+        for (int c = 0; c < 2; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float p0 = fast_exp2(fmaf(__uint_as_float(v[c * 32 + e]), p.scale_log2, -m_use));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(v[c * 32 + e + 1]), p.scale_log2, -m_use));
+            l_run += p0 + p1;
+            pk[e >> 1] = pack_bf16(p0, p1);
+          }
+          tc::tmem_st16(tS + 64 + half * 32 + c * 16, pk);
+        }
+      };
+      float mx = -INFINITY;
+      {
+        uint32_t v[64];
+        tc::tmem_ld32(tS, v);
+        tc::tmem_ld32(tS + 32, v + 32);
+        tc::tmem_wait_ld();
+        mask_half(v, 0);
+#pragma unroll
+        for (int e = 0; e < 64; ++e) mx = fmaxf(mx, __uint_as_float(v[e]));
       }
-      const bool need = m_tile > m_run + 8.f;
+      uint32_t v1[64];
+      tc::tmem_ld32(tS + 64, v1);
+      tc::tmem_ld32(tS + 96, v1 + 32);
+      tc::tmem_wait_ld();
+      mask_half(v1, 1);
+#pragma unroll
+      for (int e = 0; e < 64; ++e) mx = fmaxf(mx, __uint_as_float(v1[e]));
+      const float m_tile = mx * p.scale_log2;
+      const bool need = m_tile > m_run + kRescaleLog2;
       if (__any_sync(0xffffffffu, need)) {
         const float m_new = fmaxf(m_run, m_tile);
         const float alpha = (m_run == -INFINITY) ? 0.f : fast_exp2(m_run - m_new);
-        if (i > 0) {
+        if (t > 0) {
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
-            tc::tmem_ld32(tO + tq + c * 32, o);
+            tc::tmem_ld32(tO + c * 32, o);
             tc::tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-            tc::tmem_st32(tO + tq + c * 32, o);
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tc::tmem_st32(tO + c * 32, o);
           }
-          tc::tmem_wait_st();
         }
         l_run *= alpha;
         m_run = m_new;
       }
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      // P row -> shared memory, K-major 128-byte swizzle: chunk k of 8 keys
-#pragma unroll
-      for (int k = 0; k < kBN / 8; ++k) {
-        float pv[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          pv[e] = fast_exp2(fmaf(s[k * 8 + e], p.scale_log2, -m_use));
-          l_run += pv[e];
-        }
-        const uint32_t addr = sP + (k >> 3) * kSub + row * 128 + (((k & 7) ^ (row & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr),
-                     "r"(pack_bf16(pv[0], pv[1])), "r"(pack_bf16(pv[2], pv[3])),
-                     "r"(pack_bf16(pv[4], pv[5])), "r"(pack_bf16(pv[6], pv[7]))
-                     : "memory");
+      exp_half(v1, 1, m_use);
+      {
+        uint32_t v[64];
+        tc::tmem_ld32(tS, v);
+        tc::tmem_ld32(tS + 32, v + 32);
+        tc::tmem_wait_ld();
+        mask_half(v, 0);
+        exp_half(v, 0, m_use);
       }
-      tc::fence_async_smem();
+      tc::tmem_wait_st();
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(bar(B_PF));
+      if (lane == 0) tc::mbar_arrive(bar(B_PF + q));
     }
-    if (ok && !*abort_flag) ok = tc::mbar_wait(bar(B_OD), (nt - 1) & 1, abort_flag, p.status);
-    if (ok) {
+    const bool has_rows = my_lo <= my_hi;
+    if (ok && has_rows && !*abort_flag) ok = tc::mbar_wait(bar(B_OF + q), 0, abort_flag, p.status);
+    const uint32_t sQq = sQ + q * SM::Q_BYTES;
+    if (ok && has_rows) {
       tc::tc_fence_after();
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      // O row -> bf16 -> shared memory (the Q tile's space, same swizzled layout)
+      // O row -> bf16 -> shared memory (this tile's Q space, same swizzled layout)
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
-        tc::tmem_ld32(tO + tq + c * 32, o);
+        tc::tmem_ld32(tO + c * 32, o);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const int d8 = c * 4 + k;  // chunk of 8 columns
           const float* f = reinterpret_cast<const float*>(o + k * 8);
-          const uint32_t addr = sQ + (d8 >> 3) * kSub + row * 128 + (((d8 & 7) ^ (row & 7)) << 4);
+          const uint32_t addr = sQq + (d8 >> 3) * kSub + row * 128 + (((d8 & 7) ^ (row & 7)) << 4);
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr),
                        "r"(pack_bf16(f[0] * inv, f[1] * inv)), "r"(pack_bf16(f[2] * inv, f[3] * inv)),
                        "r"(pack_bf16(f[4] * inv, f[5] * inv)), "r"(pack_bf16(f[6] * inv, f[7] * inv))
@@ -300,16 +349,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc::fence_async_smem();
     }
-    asm volatile("bar.sync 1, 128;\n" ::: "memory");
-    if (row == 0 && ok && !*abort_flag) {
+    if (q == 0) asm volatile("bar.sync 1, 128;\n" ::: "memory");
+    else asm volatile("bar.sync 2, 128;\n" ::: "memory");
+    if (row == 0 && ok && has_rows && !*abort_flag) {
 #pragma unroll
-      for (int s = 0; s < NSUB; ++s) tc::tma_store_4d(&tmO, sQ + s * kSub, s * 64, jq, r0, b);
+      for (int s = 0; s < NSUB; ++s) tc::tma_store_4d(&tmO, sQq + s * kSub, s * 64, jq, rq0, b);
       tc::tma_store_commit_and_wait();
     }
   }
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 9) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, kTmemCols);
   }
@@ -376,7 +426,8 @@ cudaError_t launch_tc_d(const AttnParams& p, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const long long blocks = static_cast<long long>((p.Lq + kBM - 1) / kBM) * p.B * p.Hq * p.groups;
+  const long long num_qt = (p.Lq + kBM - 1) / kBM;
+  const long long blocks = (num_qt + 1) / 2 * p.B * p.Hq * p.groups;
   attn_fwd_tc_kernel<D><<<static_cast<unsigned>(blocks), kThreads, smem, stream>>>(p, mq, mk, mv, mo);
   return cudaGetLastError();
 }

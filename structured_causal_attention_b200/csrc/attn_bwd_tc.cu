@@ -35,6 +35,7 @@ namespace {
 
 constexpr int kKN = 128;   // keys per CTA
 constexpr int kQM = 64;    // query rows per iteration
+constexpr int kQS = 3;     // Q / dO stages
 constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 
@@ -45,18 +46,19 @@ struct BtSmem {
   static constexpr int QSUB = kQM * 128;    // [64 rows][64 bf16] sub-tile
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + NSUB * KSUB;
-  static constexpr int Q_OFF = V_OFF + NSUB * KSUB;          // 2 stages
-  static constexpr int DO_OFF = Q_OFF + 2 * NSUB * QSUB;     // 2 stages
-  static constexpr int P_OFF = DO_OFF + 2 * NSUB * QSUB;     // [128 keys][64 q] bf16
+  static constexpr int Q_OFF = V_OFF + NSUB * KSUB;          // kQS stages
+  static constexpr int DO_OFF = Q_OFF + kQS * NSUB * QSUB;   // kQS stages
+  static constexpr int P_OFF = DO_OFF + kQS * NSUB * QSUB;   // [128 keys][64 q] bf16
   static constexpr int DS_OFF = P_OFF + kKN * 128;
   static constexpr int DQ_OFF = DS_OFF + kKN * 128;          // D/32 boxes of [64 q][32] fp32
-  static constexpr int L_OFF = DQ_OFF + (D / 32) * kQM * 32 * 4;  // 2 stages x 64 LSE (log2)
-  static constexpr int DL_OFF = L_OFF + 2 * kQM * 4;              // 2 stages x 64 D
-  static constexpr int BAR_OFF = DL_OFF + 2 * kQM * 4;
-  static constexpr int NBAR = 15;
+  static constexpr int L_OFF = DQ_OFF + (D / 32) * kQM * 32 * 4;  // kQS stages x 64 LSE (log2)
+  static constexpr int DL_OFF = L_OFF + kQS * kQM * 4;            // kQS stages x 64 D
+  static constexpr int BAR_OFF = DL_OFF + kQS * kQM * 4;
+  static constexpr int NBAR = 16;
   static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;
   static constexpr int ABORT_OFF = SLOT_OFF + 4;
   static constexpr int USED = ABORT_OFF + 4 + 1024;
+  static_assert(USED <= 232448, "shared memory");
   // at least 120 KB: one CTA (one 512-column TMEM allocation) per SM
   static constexpr int TOTAL = USED > 120 * 1024 ? USED : 120 * 1024;
 };
@@ -64,14 +66,14 @@ struct BtSmem {
 // barrier indices
 enum {
   B_KV = 0,   // K and V loaded
-  B_QF = 1,   // [2] Q, dO and the packed LSE / D rows of a stage loaded
-  B_QE = 3,   // [2] stage free (MMA commit)
-  B_SF = 5,   // [2] S^T / dP^T ready (MMA commit)
-  B_PF = 7,   // P^T / dS^T written (4 warp arrivals)
-  B_PE = 8,   // P^T / dS^T consumed by the MMAs (MMA commit)
-  B_DF = 9,   // [2] dQ^T ready (MMA commit)
-  B_DE = 11,  // [2] dQ^T read out (4 warp arrivals)
-  B_END = 13  // every MMA done (MMA commit)
+  B_QF = 1,   // [kQS] Q, dO and the packed LSE / D rows of a stage loaded
+  B_QE = 4,   // [kQS] stage free (MMA commit)
+  B_SF = 7,   // [2] S^T / dP^T ready (MMA commit)
+  B_PF = 9,   // P^T / dS^T written (4 warp arrivals)
+  B_PE = 10,  // P^T / dS^T consumed by the MMAs (MMA commit)
+  B_DF = 11,  // [2] dQ^T ready (MMA commit)
+  B_DE = 13,  // [2] dQ^T read out (4 warp arrivals)
+  B_END = 15  // every MMA done (MMA commit)
 };
 
 template <int D>
@@ -156,8 +158,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     for (int it = 0; lane == 0 && it < total; ++it) {
-      const int st = it & 1;
-      if (!tc::mbar_wait(bar(B_QE + st), ((it >> 1) & 1) ^ 1, abort_flag, p.status)) break;
+      const int st = it % kQS;
+      if (!tc::mbar_wait(bar(B_QE + st), ((it / kQS) & 1) ^ 1, abort_flag, p.status)) break;
       const int h = iter_head(it), rq0 = iter_row0(it), jq = jq_of(h);
       if (lane == 0) {
         const long long pk = ((static_cast<long long>(b) * p.Hq + h) * p.groups + grp) * p.lq_pad + rq0;
@@ -179,15 +181,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idDQ = tc::idesc_bf16_f32(128, kQM, 1, 1);  // dQ^T
       // rows 64..127 of K^T for D = 64 read the V tile and are ignored
       constexpr uint32_t kt_lbo = (D == 64) ? (SM::V_OFF - SM::K_OFF) : SM::KSUB;
+      // Base descriptors, built once; a k-step only adds its byte offset / 16
+      // to the start-address field.
+      const uint64_t dK = tc::smem_desc_sw128(sK, 16, 1024), dV = tc::smem_desc_sw128(sV, 16, 1024);
+      const uint64_t dQk = tc::smem_desc_sw128(sQ, 16, 1024), dOk = tc::smem_desc_sw128(sDO, 16, 1024);
+      const uint64_t dQm = tc::smem_desc_sw128(sQ, SM::QSUB, 1024), dOm = tc::smem_desc_sw128(sDO, SM::QSUB, 1024);
+      const uint64_t dP = tc::smem_desc_sw128(sP, 16, 1024), dS = tc::smem_desc_sw128(sDS, 16, 1024);
+      const uint64_t dSm = tc::smem_desc_sw128(sDS, SM::QSUB, 1024);
+      const uint64_t dKt = tc::smem_desc_sw128(sK, kt_lbo, 1024);
+      auto add = [](uint64_t d, uint32_t bytes) { return d + (bytes >> 4); };
       auto issue_sp = [&](int buf, int st) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ko = (kk >> 2) * SM::KSUB + (kk & 3) * 32;
           const uint32_t qo = (st * NSUB + (kk >> 2)) * SM::QSUB + (kk & 3) * 32;
-          tc::mma_ss(tmem + 128 * buf, tc::smem_desc_sw128(sK + ko, 16, 1024),
-                     tc::smem_desc_sw128(sQ + qo, 16, 1024), idSP, kk > 0);
-          tc::mma_ss(tmem + 128 * buf + 64, tc::smem_desc_sw128(sV + ko, 16, 1024),
-                     tc::smem_desc_sw128(sDO + qo, 16, 1024), idSP, kk > 0);
+          tc::mma_ss(tmem + 128 * buf, add(dK, ko), add(dQk, qo), idSP, kk > 0);
+          tc::mma_ss(tmem + 128 * buf + 64, add(dV, ko), add(dOk, qo), idSP, kk > 0);
         }
       };
       bool ok = tc::mbar_wait(bar(B_KV), 0, abort_flag, p.status) &&
@@ -198,15 +207,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mma_commit(bar(B_SF));
       }
       for (int it = 0; ok && it < total; ++it) {
-        const int x = it & 1, st = it & 1;
+        const int x = it & 1, st = it % kQS;
         if (it + 1 < total) {
-          const int x1 = (it + 1) & 1;
-          ok = tc::mbar_wait(bar(B_QF + x1), ((it + 1) >> 1) & 1, abort_flag, p.status);
+          const int x1 = (it + 1) & 1, s1 = (it + 1) % kQS;
+          ok = tc::mbar_wait(bar(B_QF + s1), ((it + 1) / kQS) & 1, abort_flag, p.status);
           if (ok && it + 1 >= 2)
             ok = tc::mbar_wait(bar(B_DE + x1), (((it + 1) >> 1) - 1) & 1, abort_flag, p.status);
           if (!ok) break;
           tc::tc_fence_after();
-          issue_sp(x1, x1);
+          issue_sp(x1, s1);
           tc::mma_commit(bar(B_SF + x1));
         }
         ok = tc::mbar_wait(bar(B_PF), it & 1, abort_flag, p.status);
@@ -215,17 +224,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t acc = it > 0 ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < kQM / 16; ++kk) {  // reduce over the 64 queries
-          const uint64_t ap = tc::smem_desc_sw128(sP + kk * 32, 16, 1024);
-          const uint64_t as = tc::smem_desc_sw128(sDS + kk * 32, 16, 1024);
-          const uint64_t bo = tc::smem_desc_sw128(sDO + st * NSUB * SM::QSUB + kk * 2048, SM::QSUB, 1024);
-          const uint64_t bq = tc::smem_desc_sw128(sQ + st * NSUB * SM::QSUB + kk * 2048, SM::QSUB, 1024);
+          const uint64_t ap = add(dP, kk * 32);
+          const uint64_t as = add(dS, kk * 32);
+          const uint64_t bo = add(dOm, st * NSUB * SM::QSUB + kk * 2048);
+          const uint64_t bq = add(dQm, st * NSUB * SM::QSUB + kk * 2048);
           tc::mma_ss(tdV, ap, bo, idKV, (acc | kk) ? 1u : 0u);
           tc::mma_ss(tdK, as, bq, idKV, (acc | kk) ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < kKN / 16; ++kk) {  // reduce over the 128 keys
-          const uint64_t ak = tc::smem_desc_sw128(sK + kk * 2048, kt_lbo, 1024);
-          const uint64_t bs = tc::smem_desc_sw128(sDS + kk * 2048, SM::QSUB, 1024);
+          const uint64_t ak = add(dKt, kk * 2048);
+          const uint64_t bs = add(dSm, kk * 2048);
           tc::mma_ss(tmem + 128 * x, ak, bs, idDQ, kk > 0 ? 1u : 0u);
         }
         tc::mma_commit(bar(B_DF + x));
@@ -241,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tq = static_cast<uint32_t>(warp * 32) << 16;
     bool ok = true;
     for (int it = 0; it < total; ++it) {
-      const int x = it & 1, st = it & 1;
+      const int x = it & 1, st = it % kQS;
       const int rq0 = iter_row0(it);
       if (!tc::mbar_wait(bar(B_SF + x), (it >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
       tc::tc_fence_after();
@@ -256,22 +265,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tmem_ld32(tmem + tq + 128 * x + 64 + half * 32, dr);
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          float pj[2], dj[2];
+        for (int j = 0; j < 32; j += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(sL + st * kQM + half * 32 + j);
+          const float4 d4 = *reinterpret_cast<const float4*>(sDl + st * kQM + half * 32 + j);
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+          const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+          float pj[4], dj[4];
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
+          for (int e = 0; e < 4; ++e) {
             const int rl = half * 32 + j + e;
-            float pv = fast_exp2(fmaf(__uint_as_float(sr[j + e]), p.scale_log2, -sL[st * kQM + rl]));
+            float pv = fast_exp2(fmaf(__uint_as_float(sr[j + e]), p.scale_log2, -lv[e]));
             if (!full) {
               const int r = rq0 + rl;
               const int hi = p.a * r + p.bb;
               if (!(r < p.Lq && c <= hi && c > hi - p.win && c < p.Lk)) pv = 0.f;
             }
             pj[e] = pv;
-            dj[e] = pv * (__uint_as_float(dr[j + e]) - sDl[st * kQM + rl]);
+            dj[e] = pv * (__uint_as_float(dr[j + e]) - dv4[e]);
           }
           pp[half * 16 + j / 2] = pack_bf16(pj[0], pj[1]);
+          pp[half * 16 + j / 2 + 1] = pack_bf16(pj[2], pj[3]);
           dd[half * 16 + j / 2] = pack_bf16(dj[0], dj[1]);
+          dd[half * 16 + j / 2 + 1] = pack_bf16(dj[2], dj[3]);
         }
       }
       // the MMAs of the previous tile have finished reading P^T / dS^T

@@ -13,15 +13,18 @@
 //   dV  += P^T dO     (M 128 keys, N D)            } accumulated in TMEM across
 //   dK  += dS^T Q     (M 128 keys, N D)            } the whole group
 //   dQ^T = K^T dS^T   (M D, N 64 queries)           into the S^T buffer
-// Roles (10 warps):
-//   warps 0-3   one key row per thread: P^T = exp2(S^T - LSE), dS^T = P^T (dP^T - D),
+// Roles (14 warps):
+//   warps 0-7   two warpgroups, one key row per thread, each taking 32 of the
+//               64 query columns: P^T = exp2(S^T - LSE), dS^T = P^T (dP^T - D),
 //               written as bf16 into shared memory in the MMA operand layout;
-//               at the end dK (scaled) and dV go out through TMA stores.
-//   warps 4-7   one head-dim row per thread: dQ^T from TMEM into an fp32 tile,
-//               added into the fp32 dQ accumulator with a TMA bulk reduce-add.
-//   warp 8      TMA: K, V once; Q and dO tiles (2 stages) plus the tile's
+//               at the end warpgroup 0 stores dK (scaled) and warpgroup 1 dV
+//               through TMA.
+//   warps 8-11  one head-dim row per thread: dQ^T from TMEM, added into the
+//               fp32 dQ accumulator with coalesced reductions (each warp
+//               covers 32 consecutive head-dim entries of a query row).
+//   warp 12     TMA: K, V once; Q and dO tiles (3 stages) plus the tile's
 //               packed LSE and D rows (bulk copies).
-//   warp 9      TMEM allocation; lane 0 issues the MMAs.
+//   warp 13     TMEM allocation; lane 0 issues the MMAs.
 // Every mbarrier wait is bounded (HD_ERR_TIMEOUT, then every role leaves).
 #include <cuda.h>
 
@@ -36,7 +39,7 @@ namespace {
 constexpr int kKN = 128;   // keys per CTA
 constexpr int kQM = 64;    // query rows per iteration
 constexpr int kQS = 3;     // Q / dO stages
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;
 constexpr uint32_t kTmemCols = 512;
 
 template <int D>
@@ -50,8 +53,7 @@ struct BtSmem {
   static constexpr int DO_OFF = Q_OFF + kQS * NSUB * QSUB;   // kQS stages
   static constexpr int P_OFF = DO_OFF + kQS * NSUB * QSUB;   // [128 keys][64 q] bf16
   static constexpr int DS_OFF = P_OFF + kKN * 128;
-  static constexpr int DQ_OFF = DS_OFF + kKN * 128;          // D/32 boxes of [64 q][32] fp32
-  static constexpr int L_OFF = DQ_OFF + (D / 32) * kQM * 32 * 4;  // kQS stages x 64 LSE (log2)
+  static constexpr int L_OFF = DS_OFF + kKN * 128;           // kQS stages x 64 LSE (log2)
   static constexpr int DL_OFF = L_OFF + kQS * kQM * 4;            // kQS stages x 64 D
   static constexpr int BAR_OFF = DL_OFF + kQS * kQM * 4;
   static constexpr int NBAR = 16;
@@ -69,7 +71,7 @@ enum {
   B_QF = 1,   // [kQS] Q, dO and the packed LSE / D rows of a stage loaded
   B_QE = 4,   // [kQS] stage free (MMA commit)
   B_SF = 7,   // [2] S^T / dP^T ready (MMA commit)
-  B_PF = 9,   // P^T / dS^T written (4 warp arrivals)
+  B_PF = 9,   // P^T / dS^T written (8 warp arrivals)
   B_PE = 10,  // P^T / dS^T consumed by the MMAs (MMA commit)
   B_DF = 11,  // [2] dQ^T ready (MMA commit)
   B_DE = 13,  // [2] dQ^T read out (4 warp arrivals)
@@ -81,15 +83,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDK,
-                       const __grid_constant__ CUtensorMap tmDV, const __grid_constant__ CUtensorMap tmDQ) {
+                       const __grid_constant__ CUtensorMap tmDV) {
   using SM = BtSmem<D>;
   constexpr int NSUB = SM::NSUB;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
   const uint32_t sK = sbase + SM::K_OFF, sV = sbase + SM::V_OFF, sQ = sbase + SM::Q_OFF,
-                 sDO = sbase + SM::DO_OFF, sP = sbase + SM::P_OFF, sDS = sbase + SM::DS_OFF,
-                 sDQ = sbase + SM::DQ_OFF;
+                 sDO = sbase + SM::DO_OFF, sP = sbase + SM::P_OFF, sDS = sbase + SM::DS_OFF;
   float* sL = reinterpret_cast<float*>(sgen + SM::L_OFF);
   float* sDl = reinterpret_cast<float*>(sgen + SM::DL_OFF);
   auto bar = [&](int i) { return sbase + SM::BAR_OFF + 8u * i; };
@@ -127,13 +128,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < SM::NBAR; ++i) {
       uint32_t cnt = 1;
-      if (i == B_PF || i == B_DE || i == B_DE + 1) cnt = 4;
+      if (i == B_DE || i == B_DE + 1) cnt = 4;
+      if (i == B_PF) cnt = 8;
       tc::mbar_init(bar(i), cnt);
     }
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tc::tmem_alloc(sbase + SM::SLOT_OFF, kTmemCols);
     tc::tmem_relinquish();
   }
@@ -145,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // dK at 256, dV at 256 + D.
   const uint32_t tdK = tmem + 256, tdV = tmem + 256 + D;
 
-  if (warp == 8) {
+  if (warp == 12) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tc::tma_prefetch_desc(&tmQ);
@@ -173,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::bulk_load(sbase + SM::DL_OFF + st * kQM * 4, p.deltap + pk, kQM * 4, bar(B_QF + st));
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0 && total > 0) {
       constexpr uint32_t idSP = tc::idesc_bf16_f32(128, kQM, 0, 0);  // S^T, dP^T
@@ -243,11 +245,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc::mma_commit(bar(B_END));
     }
-  } else if (warp < 4) {
-    // ------------------------------------------------ P^T, dS^T (one key per thread)
-    const int row = tid;
+  } else if (warp < 8) {
+    // ------------------------- P^T, dS^T: one key per thread, warpgroup sw takes
+    // query columns 32*sw .. 32*sw+31
+    const int sw = warp >> 2;
+    const int row = tid & 127;
     const int c = c0 + row;
-    const uint32_t tq = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tq = static_cast<uint32_t>((warp & 3) * 32) << 16;
     bool ok = true;
     for (int it = 0; it < total; ++it) {
       const int x = it & 1, st = it % kQS;
@@ -257,36 +261,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool full = (c0 + kKN - 1 <= p.a * rq0 + p.bb) &&
                         (c0 > p.a * (rq0 + kQM - 1) + p.bb - p.win) && (c0 + kKN <= p.Lk) &&
                         (rq0 + kQM <= p.Lq);
-      uint32_t pp[32], dd[32];  // bf16 pairs of P^T and dS^T for the 64 queries
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      uint32_t pp[16], dd[16];  // bf16 pairs of P^T and dS^T for this warpgroup's 32 queries
+      {
         uint32_t sr[32], dr[32];
-        tc::tmem_ld32(tmem + tq + 128 * x + half * 32, sr);
-        tc::tmem_ld32(tmem + tq + 128 * x + 64 + half * 32, dr);
+        tc::tmem_ld32(tmem + tq + 128 * x + sw * 32, sr);
+        tc::tmem_ld32(tmem + tq + 128 * x + 64 + sw * 32, dr);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(sL + st * kQM + half * 32 + j);
-          const float4 d4 = *reinterpret_cast<const float4*>(sDl + st * kQM + half * 32 + j);
+          const float4 l4 = *reinterpret_cast<const float4*>(sL + st * kQM + sw * 32 + j);
+          const float4 d4 = *reinterpret_cast<const float4*>(sDl + st * kQM + sw * 32 + j);
           const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
           const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
           float pj[4], dj[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int rl = half * 32 + j + e;
             float pv = fast_exp2(fmaf(__uint_as_float(sr[j + e]), p.scale_log2, -lv[e]));
             if (!full) {
-              const int r = rq0 + rl;
+              const int r = rq0 + sw * 32 + j + e;
               const int hi = p.a * r + p.bb;
               if (!(r < p.Lq && c <= hi && c > hi - p.win && c < p.Lk)) pv = 0.f;
             }
             pj[e] = pv;
             dj[e] = pv * (__uint_as_float(dr[j + e]) - dv4[e]);
           }
-          pp[half * 16 + j / 2] = pack_bf16(pj[0], pj[1]);
-          pp[half * 16 + j / 2 + 1] = pack_bf16(pj[2], pj[3]);
-          dd[half * 16 + j / 2] = pack_bf16(dj[0], dj[1]);
-          dd[half * 16 + j / 2 + 1] = pack_bf16(dj[2], dj[3]);
+          pp[j / 2] = pack_bf16(pj[0], pj[1]);
+          pp[j / 2 + 1] = pack_bf16(pj[2], pj[3]);
+          dd[j / 2] = pack_bf16(dj[0], dj[1]);
+          dd[j / 2 + 1] = pack_bf16(dj[2], dj[3]);
         }
       }
       // the MMAs of the previous tile have finished reading P^T / dS^T
@@ -294,13 +296,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!tc::mbar_wait(bar(B_PE), (it - 1) & 1, abort_flag, p.status)) { ok = false; break; }
       }
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
+      for (int k = 0; k < 4; ++k) {
+        const int ch = sw * 4 + k;
         const uint32_t off = row * 128 + ((ch ^ (row & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(sP + off), "r"(pp[4 * ch]),
-                     "r"(pp[4 * ch + 1]), "r"(pp[4 * ch + 2]), "r"(pp[4 * ch + 3])
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(sP + off), "r"(pp[4 * k]),
+                     "r"(pp[4 * k + 1]), "r"(pp[4 * k + 2]), "r"(pp[4 * k + 3])
                      : "memory");
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(sDS + off), "r"(dd[4 * ch]),
-                     "r"(dd[4 * ch + 1]), "r"(dd[4 * ch + 2]), "r"(dd[4 * ch + 3])
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(sDS + off), "r"(dd[4 * k]),
+                     "r"(dd[4 * k + 1]), "r"(dd[4 * k + 2]), "r"(dd[4 * k + 3])
                      : "memory");
       }
       tc::fence_async_smem();
@@ -308,52 +311,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(bar(B_PF));
     }
-    // ---- dK (scaled), dV: TMEM -> bf16 -> shared memory (Q / dO stages) -> TMA store
+    // ---- warpgroup 0: dK (scaled), warpgroup 1: dV; TMEM -> bf16 -> shared
+    // memory (the Q / dO stages) -> TMA store
     if (ok && !*abort_flag && total > 0) ok = tc::mbar_wait(bar(B_END), 0, abort_flag, p.status);
+    const uint32_t src = sw == 0 ? tdK : tdV;
+    const uint32_t dst = sw == 0 ? sQ : sDO;  // kQS x NSUB x [64][64] >= NSUB x [128][64]
+    const float sc = sw == 0 ? p.scale : 1.f;
     if (ok && !*abort_flag) {
       tc::tc_fence_after();
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const uint32_t src = t == 0 ? tdK : tdV;
-        const uint32_t dst = t == 0 ? sQ : sDO;  // 2 stages x NSUB x [64][64] = NSUB x [128][64]
-        const float sc = t == 0 ? p.scale : 1.f;
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t v[32];
+        if (total > 0) {
+          tc::tmem_ld32(src + tq + cc * 32, v);
+          tc::tmem_wait_ld();
+        } else {
 #pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t v[32];
-          if (total > 0) {
-            tc::tmem_ld32(src + tq + cc * 32, v);
-            tc::tmem_wait_ld();
-          } else {
+          for (int j = 0; j < 32; ++j) v[j] = 0u;
+        }
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = 0u;
-          }
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int d8 = cc * 4 + k;
-            const float* f = reinterpret_cast<const float*>(v + 8 * k);
-            const uint32_t addr = dst + (d8 >> 3) * SM::KSUB + row * 128 + (((d8 & 7) ^ (row & 7)) << 4);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr),
-                         "r"(pack_bf16(f[0] * sc, f[1] * sc)), "r"(pack_bf16(f[2] * sc, f[3] * sc)),
-                         "r"(pack_bf16(f[4] * sc, f[5] * sc)), "r"(pack_bf16(f[6] * sc, f[7] * sc))
-                         : "memory");
-          }
+        for (int k = 0; k < 4; ++k) {
+          const int d8 = cc * 4 + k;
+          const float* f = reinterpret_cast<const float*>(v + 8 * k);
+          const uint32_t addr = dst + (d8 >> 3) * SM::KSUB + row * 128 + (((d8 & 7) ^ (row & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr),
+                       "r"(pack_bf16(f[0] * sc, f[1] * sc)), "r"(pack_bf16(f[2] * sc, f[3] * sc)),
+                       "r"(pack_bf16(f[4] * sc, f[5] * sc)), "r"(pack_bf16(f[6] * sc, f[7] * sc))
+                       : "memory");
         }
       }
       tc::fence_async_smem();
     }
-    asm volatile("bar.sync 1, 128;\n" ::: "memory");
+    if (sw == 0) asm volatile("bar.sync 1, 128;\n" ::: "memory");
+    else asm volatile("bar.sync 2, 128;\n" ::: "memory");
     if (row == 0 && ok && !*abort_flag) {
 #pragma unroll
-      for (int s = 0; s < NSUB; ++s) {
-        tc::tma_store_4d(&tmDK, sQ + s * SM::KSUB, s * 64, jk, c0, b);
-        tc::tma_store_4d(&tmDV, sDO + s * SM::KSUB, s * 64, jk, c0, b);
-      }
+      for (int s = 0; s < NSUB; ++s) tc::tma_store_4d(sw == 0 ? &tmDK : &tmDV, dst + s * SM::KSUB, s * 64, jk, c0, b);
       tc::tma_store_commit_and_wait();
     }
-  } else {
-    // ------------------------------------- dQ^T readout (one head-dim row per thread)
-    const int d = tid - 128;
-    const uint32_t tq = static_cast<uint32_t>((warp - 4) * 32) << 16;
+  } else if (warp < 12) {
+    // ------------------- dQ^T read-out (one head-dim row per thread), added into
+    // the fp32 accumulator with coalesced reductions (32 consecutive d per warp)
+    const int d = tid - 256;
+    const uint32_t tq = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const long long q_row0 = static_cast<long long>(b) * p.Sq + static_cast<long long>(grp) * p.qs_step;
+    const long long q_rs = static_cast<long long>(p.q_rstride) * p.Hq * D;
     for (int it = 0; it < total; ++it) {
       const int x = it & 1;
       if (!tc::mbar_wait(bar(B_DF + x), (it >> 1) & 1, abort_flag, p.status)) break;
@@ -365,35 +367,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(bar(B_DE + x));
-      // the previous reduce-add has finished reading the staging tile
-      if (d == 0) asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
-      asm volatile("bar.sync 2, 128;\n" ::: "memory");
       if (d < D) {
-        float* stg = reinterpret_cast<float*>(sgen + SM::DQ_OFF) + (d >> 5) * (kQM * 32) + (d & 31);
+        const int h = iter_head(it), rq0 = iter_row0(it);
+        float* base = p.dq_acc + (q_row0 * p.Hq + h) * D + d + static_cast<long long>(rq0) * q_rs;
+        const int nq = min(kQM, p.Lq - rq0);
 #pragma unroll
-        for (int q = 0; q < 32; ++q) stg[q * 32] = __uint_as_float(v0[q]);
+        for (int q = 0; q < 32; ++q)
+          if (q < nq) atomicAdd(base + q * q_rs, __uint_as_float(v0[q]));
 #pragma unroll
-        for (int q = 0; q < 32; ++q) stg[(q + 32) * 32] = __uint_as_float(v1[q]);
-      }
-      tc::fence_async_smem();
-      asm volatile("bar.sync 2, 128;\n" ::: "memory");
-      if (d == 0) {
-        const int h = iter_head(it), rq0 = iter_row0(it), jq = jq_of(h);
-#pragma unroll
-        for (int bx = 0; bx < D / 32; ++bx)
-          asm volatile(
-              "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group"
-              " [%0, {%2, %3, %4, %5}], [%1];\n" ::"l"(reinterpret_cast<uint64_t>(&tmDQ)),
-              "r"(sDQ + bx * kQM * 32 * 4), "r"(bx * 32), "r"(jq), "r"(rq0), "r"(b)
-              : "memory");
-        asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
+        for (int q = 0; q < 32; ++q)
+          if (q + 32 < nq) atomicAdd(base + (q + 32) * q_rs, __uint_as_float(v1[q]));
       }
     }
-    if (d == 0) asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
   }
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, kTmemCols);
   }
@@ -440,7 +429,7 @@ bool make_map(CUtensorMap* map, const void* base, bool fp32, int D, long long J,
 template <int D>
 cudaError_t launch_bwd_tc_d(const AttnParams& p, cudaStream_t stream) {
   const long long S = p.S, L = p.L, n = p.n, Hq = p.Hq, Hkv = p.Hkv, B = p.B;
-  CUtensorMap mq, mdo, mk, mv, mdk, mdv, mdq;
+  CUtensorMap mq, mdo, mk, mv, mdk, mdv;
   const bool intra = p.mode == HD_INTRA;
   long long Jq, Rq, sjq, srq, sbq;
   if (intra && !p.final_only) {
@@ -456,7 +445,6 @@ cudaError_t launch_bwd_tc_d(const AttnParams& p, cudaStream_t stream) {
   }
   bool ok = make_map(&mq, p.q, false, D, Jq, Rq, B, sjq, srq, sbq, 64, kQM) &&
             make_map(&mdo, p.dout, false, D, Jq, Rq, B, sjq, srq, sbq, 64, kQM) &&
-            make_map(&mdq, p.dq_acc, true, D, Jq, Rq, B, sjq, srq, sbq, 32, kQM) &&
             make_map(&mk, p.k, false, D, Jk, Rk, B, D, srk, sbk, 64, kKN) &&
             make_map(&mv, p.v, false, D, Jk, Rk, B, D, srk, sbk, 64, kKN) &&
             make_map(&mdk, p.dk, false, D, Jk, Rk, B, D, srk, sbk, 64, kKN) &&
@@ -468,7 +456,7 @@ cudaError_t launch_bwd_tc_d(const AttnParams& p, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   const long long blocks = static_cast<long long>((p.Lk + kKN - 1) / kKN) * p.B * p.Hkv * p.groups;
   attn_bwd_tc_kernel<D><<<static_cast<unsigned>(blocks), kThreads, smem, stream>>>(p, mq, mdo, mk, mv,
-                                                                                   mdk, mdv, mdq);
+                                                                                   mdk, mdv);
   return cudaGetLastError();
 }
 

@@ -19,9 +19,9 @@
 //               written as bf16 into shared memory in the MMA operand layout;
 //               at the end warpgroup 0 stores dK (scaled) and warpgroup 1 dV
 //               through TMA.
-//   warps 8-11  one head-dim row per thread: dQ^T from TMEM, added into the
-//               fp32 dQ accumulator with coalesced reductions (each warp
-//               covers 32 consecutive head-dim entries of a query row).
+//   warps 8-11  one head-dim row per thread: dQ^T from TMEM into an fp32 tile
+//               in shared memory, added into the fp32 dQ accumulator by a TMA
+//               bulk reduce-add (the TMA unit does the adds, not the SM).
 //   warp 12     TMA: K, V once; Q and dO tiles (3 stages) plus the tile's
 //               packed LSE and D rows (bulk copies).
 //   warp 13     TMEM allocation; lane 0 issues the MMAs.
@@ -53,7 +53,8 @@ struct BtSmem {
   static constexpr int DO_OFF = Q_OFF + kQS * NSUB * QSUB;   // kQS stages
   static constexpr int P_OFF = DO_OFF + kQS * NSUB * QSUB;   // [128 keys][64 q] bf16
   static constexpr int DS_OFF = P_OFF + kKN * 128;
-  static constexpr int L_OFF = DS_OFF + kKN * 128;           // kQS stages x 64 LSE (log2)
+  static constexpr int DQ_OFF = DS_OFF + kKN * 128;          // D/32 boxes of [64 q][32] fp32
+  static constexpr int L_OFF = DQ_OFF + (D / 32) * kQM * 32 * 4;  // kQS stages x 64 LSE (log2)
   static constexpr int DL_OFF = L_OFF + kQS * kQM * 4;            // kQS stages x 64 D
   static constexpr int BAR_OFF = DL_OFF + kQS * kQM * 4;
   static constexpr int NBAR = 16;
@@ -83,14 +84,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDK,
-                       const __grid_constant__ CUtensorMap tmDV) {
+                       const __grid_constant__ CUtensorMap tmDV, const __grid_constant__ CUtensorMap tmDQ) {
   using SM = BtSmem<D>;
   constexpr int NSUB = SM::NSUB;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
   const uint32_t sK = sbase + SM::K_OFF, sV = sbase + SM::V_OFF, sQ = sbase + SM::Q_OFF,
-                 sDO = sbase + SM::DO_OFF, sP = sbase + SM::P_OFF, sDS = sbase + SM::DS_OFF;
+                 sDO = sbase + SM::DO_OFF, sP = sbase + SM::P_OFF, sDS = sbase + SM::DS_OFF,
+                 sDQ = sbase + SM::DQ_OFF;
   float* sL = reinterpret_cast<float*>(sgen + SM::L_OFF);
   float* sDl = reinterpret_cast<float*>(sgen + SM::DL_OFF);
   auto bar = [&](int i) { return sbase + SM::BAR_OFF + 8u * i; };
@@ -354,8 +356,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the fp32 accumulator with coalesced reductions (32 consecutive d per warp)
     const int d = tid - 256;
     const uint32_t tq = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const long long q_row0 = static_cast<long long>(b) * p.Sq + static_cast<long long>(grp) * p.qs_step;
-    const long long q_rs = static_cast<long long>(p.q_rstride) * p.Hq * D;
     for (int it = 0; it < total; ++it) {
       const int x = it & 1;
       if (!tc::mbar_wait(bar(B_DF + x), (it >> 1) & 1, abort_flag, p.status)) break;
@@ -367,18 +367,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(bar(B_DE + x));
+      // the previous reduce-add has finished reading the staging tile
+      if (d == 0) asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
+      asm volatile("bar.sync 3, 128;\n" ::: "memory");
       if (d < D) {
-        const int h = iter_head(it), rq0 = iter_row0(it);
-        float* base = p.dq_acc + (q_row0 * p.Hq + h) * D + d + static_cast<long long>(rq0) * q_rs;
-        const int nq = min(kQM, p.Lq - rq0);
+        float* stg = reinterpret_cast<float*>(sgen + SM::DQ_OFF) + (d >> 5) * (kQM * 32) + (d & 31);
 #pragma unroll
-        for (int q = 0; q < 32; ++q)
-          if (q < nq) atomicAdd(base + q * q_rs, __uint_as_float(v0[q]));
+        for (int q = 0; q < 32; ++q) stg[q * 32] = __uint_as_float(v0[q]);
 #pragma unroll
-        for (int q = 0; q < 32; ++q)
-          if (q + 32 < nq) atomicAdd(base + (q + 32) * q_rs, __uint_as_float(v1[q]));
+        for (int q = 0; q < 32; ++q) stg[(q + 32) * 32] = __uint_as_float(v1[q]);
+      }
+      tc::fence_async_smem();
+      asm volatile("bar.sync 3, 128;\n" ::: "memory");
+      if (d == 0) {
+        const int h = iter_head(it), rq0 = iter_row0(it), jq = jq_of(h);
+#pragma unroll
+        for (int bx = 0; bx < D / 32; ++bx)
+          asm volatile(
+              "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group"
+              " [%0, {%2, %3, %4, %5}], [%1];\n" ::"l"(reinterpret_cast<uint64_t>(&tmDQ)),
+              "r"(sDQ + bx * kQM * 32 * 4), "r"(bx * 32), "r"(jq), "r"(rq0), "r"(b)
+              : "memory");
+        asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
       }
     }
+    if (d == 0) asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -429,7 +442,7 @@ bool make_map(CUtensorMap* map, const void* base, bool fp32, int D, long long J,
 template <int D>
 cudaError_t launch_bwd_tc_d(const AttnParams& p, cudaStream_t stream) {
   const long long S = p.S, L = p.L, n = p.n, Hq = p.Hq, Hkv = p.Hkv, B = p.B;
-  CUtensorMap mq, mdo, mk, mv, mdk, mdv;
+  CUtensorMap mq, mdo, mk, mv, mdk, mdv, mdq;
   const bool intra = p.mode == HD_INTRA;
   long long Jq, Rq, sjq, srq, sbq;
   if (intra && !p.final_only) {
@@ -445,6 +458,7 @@ cudaError_t launch_bwd_tc_d(const AttnParams& p, cudaStream_t stream) {
   }
   bool ok = make_map(&mq, p.q, false, D, Jq, Rq, B, sjq, srq, sbq, 64, kQM) &&
             make_map(&mdo, p.dout, false, D, Jq, Rq, B, sjq, srq, sbq, 64, kQM) &&
+            make_map(&mdq, p.dq_acc, true, D, Jq, Rq, B, sjq, srq, sbq, 32, kQM) &&
             make_map(&mk, p.k, false, D, Jk, Rk, B, D, srk, sbk, 64, kKN) &&
             make_map(&mv, p.v, false, D, Jk, Rk, B, D, srk, sbk, 64, kKN) &&
             make_map(&mdk, p.dk, false, D, Jk, Rk, B, D, srk, sbk, 64, kKN) &&
@@ -456,7 +470,7 @@ cudaError_t launch_bwd_tc_d(const AttnParams& p, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   const long long blocks = static_cast<long long>((p.Lk + kKN - 1) / kKN) * p.B * p.Hkv * p.groups;
   attn_bwd_tc_kernel<D><<<static_cast<unsigned>(blocks), kThreads, smem, stream>>>(p, mq, mdo, mk, mv,
-                                                                                   mdk, mdv);
+                                                                                   mdk, mdv, mdq);
   return cudaGetLastError();
 }
 

@@ -269,6 +269,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tmem_ld32(tmem + tq + 128 * x + sw * 32, sr);
         tc::tmem_ld32(tmem + tq + 128 * x + 64 + sw * 32, dr);
         tc::tmem_wait_ld();
+        // The mask is a separate pass (score -> -inf, so P and dS become 0):
+        // a test inside the arithmetic loop below would serialise it.
+        if (!full) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int r = rq0 + sw * 32 + e;
+            const int hi = p.a * r + p.bb;
+            if (!(r < p.Lq && c <= hi && c > hi - p.win && c < p.Lk)) sr[e] = __float_as_uint(-INFINITY);
+          }
+        }
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
           const float4 l4 = *reinterpret_cast<const float4*>(sL + st * kQM + sw * 32 + j);
@@ -278,12 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float pj[4], dj[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            float pv = fast_exp2(fmaf(__uint_as_float(sr[j + e]), p.scale_log2, -lv[e]));
-            if (!full) {
-              const int r = rq0 + sw * 32 + j + e;
-              const int hi = p.a * r + p.bb;
-              if (!(r < p.Lq && c <= hi && c > hi - p.win && c < p.Lk)) pv = 0.f;
-            }
+            const float pv = fast_exp2(fmaf(__uint_as_float(sr[j + e]), p.scale_log2, -lv[e]));
             pj[e] = pv;
             dj[e] = pv * (__uint_as_float(dr[j + e]) - dv4[e]);
           }

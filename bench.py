@@ -374,11 +374,7 @@ DESCRIPTIONS = {
 # DRAM bytes per launch of the dominant kernel from the last ncu capture of
 # the same build (dram__bytes_read.sum + dram__bytes_write.sum); None when the
 # kernel changed after that capture.
-NCU_TRAFFIC = {
-    # attn_bwd_tc_kernel, CROSS_FULL at the intra_train sizes (profiles/
-    # attn_bwd_tc_kernel_cross_full_intra_train.md): 2.821 GB read + 1.437 GB written
-    ("step", "bwd_cross_full"): 4257670000,
-}
+NCU_TRAFFIC = {}
 
 
 def main():

@@ -27,3 +27,4 @@ from .attention import (  # noqa: F401
 )
 from .decode import decode_attn  # noqa: F401
 from .expand import expand_embed  # noqa: F401
+from .rope import rope, rope_expanded  # noqa: F401

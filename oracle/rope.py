@@ -35,9 +35,22 @@ def rope(x, positions, base):
     return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
 
 
-def rope_expanded(q, k, n, final_only, base):
-    """RoPE of q (all positions, or final-stream rows) and k at physical positions."""
+def rope_expanded(q, k, n, final_only, base, token_offset=None):
+    """RoPE of q (all positions, or final-stream rows) and k at physical positions.
+
+    token_offset[b] tokens precede the rows of sequence b, shifting every
+    position of that sequence by token_offset[b] * n (a decode step).
+    """
+    ref = k if k is not None else q
+    B = ref.shape[0]
     S = k.shape[1] if k is not None else (q.shape[1] * (n if final_only else 1))
-    out_q = rope(q, query_positions(S, n, final_only), base) if q is not None else None
-    out_k = rope(k, np.arange(S), base) if k is not None else None
+    offs = np.zeros(B, dtype=np.int64) if token_offset is None else np.asarray(token_offset, np.int64)
+    out_q = np.empty(q.shape) if q is not None else None
+    out_k = np.empty(k.shape) if k is not None else None
+    for b in range(B):
+        shift = int(offs[b]) * n
+        if q is not None:
+            out_q[b:b + 1] = rope(q[b:b + 1], query_positions(S, n, final_only) + shift, base)
+        if k is not None:
+            out_k[b:b + 1] = rope(k[b:b + 1], np.arange(S) + shift, base)
     return out_q, out_k

@@ -72,3 +72,19 @@ def test_expanded_positions_are_physical(n):
     if n > 1:  # a token index instead of the physical position would differ
         tok = oracle.rope(q[:, 1:2], [0], 10000.0)
         assert np.abs(tok - oq[:, 1:2]).max() > 1e-3
+
+
+def test_token_offset_matches_the_tail_of_a_longer_sequence():
+    """A decode step at offset T sees the positions of token T of a T+1-token prefill."""
+    n, T, H, D = 3, 6, 2, 16
+    k = _rand((2, (T + 1) * n, H, D), 7)
+    q = _rand((2, T + 1, H, D), 8)
+    fq, fk = oracle.rope_expanded(q, k, n, True, 10000.0)
+    dq, dk = oracle.rope_expanded(q[:, T:], k[:, T * n:], n, True, 10000.0, token_offset=[T, T])
+    np.testing.assert_array_equal(dk, fk[:, T * n:])
+    np.testing.assert_array_equal(dq, fq[:, T:])
+    # per-sequence offsets are independent
+    mixed = np.stack([q[0, T:T + 1], q[1, 0:1]])
+    mq, _ = oracle.rope_expanded(mixed, None, n, True, 10000.0, token_offset=[T, 0])
+    np.testing.assert_array_equal(mq[0, 0], fq[0, T])
+    np.testing.assert_array_equal(mq[1, 0], fq[1, 0])

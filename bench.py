@@ -87,10 +87,14 @@ def step_plan(wl):
                         pairs=pr, bytes=kv_bytes + io))
     ex_bytes = B * L * 4 + 2 * B * L * n * wl["d"] * 4
     ops.insert(0, dict(name="expand", kind="expand", flops=0, pairs=0, bytes=ex_bytes))
+    # rotary embedding of q and k in place: every element read and written once
+    ops.append(dict(name="rope", kind="rope", flops=0, pairs=0, bytes=2 * 2 * B * S * (Hq + Hkv) * D))
     return ops
 
 
-LAUNCHES = {"expand": 1, "fwd": 1, "bwd": 3, "decode": 2}
+LAUNCHES = {"expand": 1, "fwd": 1, "bwd": 3, "decode": 2, "rope": 1}
+# operations measured on their own only (not part of the default hot-path step)
+EXTRA_KINDS = {"rope"}
 
 # Extra workloads for per-configuration measurements (`--workload`); the
 # default is the whole hot-path step above.
@@ -108,6 +112,8 @@ WORKLOADS = {
                      ops=["decode_cross_full", "decode_intra"]),
     "expand": dict(B=4, L=8192, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=1,
                    ops=["expand"]),
+    "rope": dict(B=1, L=32768, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=1,
+                 ops=["rope"]),
 }
 
 
@@ -116,6 +122,8 @@ def plan_for(name):
     ops = step_plan(wl)
     if wl["ops"] is not None:
         ops = [o for o in ops if o["name"] in wl["ops"]]
+    else:
+        ops = [o for o in ops if o["kind"] not in EXTRA_KINDS]
     return wl, ops
 
 
@@ -155,6 +163,9 @@ class Step:
                     self.h["dof"] = syn.normal_bf16((B, L, Hq, D), 13)
         if "decode" in kinds:
             self.h["dq_new"] = syn.normal_bf16((B, n, Hq, D), 14)
+        if "rope" in kinds and not attn:
+            self.h["q"] = syn.normal_bf16((B, S, Hq, D), 16)
+            self.h["k"] = syn.normal_bf16((B, S, Hkv, D), 17)
         for k_ in list(self.h):
             self.h[k_] = self.h[k_].pin_memory()
         self.d = {k_: v_.to(dev) for k_, v_ in self.h.items()}
@@ -199,6 +210,8 @@ class Step:
             self.result.append(next(iter(self.lse.values())))
         elif "expand" in kinds:
             self.result.append(self.x[:, :1])
+        elif "rope" in kinds:
+            self.result.append(self.d["k"][:, :1])
         self.host_res = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in self.result]
         self.d2h_bytes = sum(t.numel() * t.element_size() for t in self.result)
 
@@ -210,6 +223,8 @@ class Step:
         name = op["name"]
         if op["kind"] == "expand":
             hd.hd_expand_embed(d["ids"], self.tables, self.x, B, L, n, wl["V"], wl["d"], 4, s)
+        elif op["kind"] == "rope":
+            hd.hd_rope_expanded(d["q"], d["k"], None, B, L, n, Hq, Hkv, D, 0, 10000.0, s)
         elif op["kind"] in ("fwd", "bwd"):
             key = name.split("_", 1)[1]
             fin = op["fin"]
@@ -369,6 +384,7 @@ DESCRIPTIONS = {
     "decode8": "decode step CROSS_FULL + INTRA, B8 n4, 16384 prior tokens (65540 cache rows), Hq32 Hkv8 D128",
     "decode64": "decode step CROSS_FULL + INTRA, B64 n4, 16384 prior tokens (65540 cache rows), Hq32 Hkv8 D128",
     "expand": "expansion B4 L8192 n4, V32000, d4096 fp32 tables",
+    "rope": "RoPE in place at physical positions, q [1,131072,32,128] + k [1,131072,8,128] bf16, base 10000",
 }
 
 # DRAM bytes per launch of the dominant kernel from the last ncu capture of
@@ -393,7 +409,7 @@ def main():
     wl, ops = plan_for(args.workload)
     total_flops = sum(o["flops"] for o in ops)
     total_bytes = sum(o.get("bytes", 0) for o in ops)
-    hbm_only = total_flops == 0 or all(o["kind"] in ("decode", "expand") for o in ops)
+    hbm_only = total_flops == 0 or all(o["kind"] in ("decode", "expand", "rope") for o in ops)
     tokens = wl["B"] * wl["n"] * wl["L"]
     config = {"workload": DESCRIPTIONS[args.workload],
               "global_batch": wl["B"] * max(world, 1), "seq_len": wl["n"] * wl["L"],
@@ -542,7 +558,8 @@ def main():
     kname = {"fwd": "hd_attn_fwd (attn_fwd_tc_kernel)",
              "bwd": "hd_attn_bwd (bwd_pre + attn_bwd_tc_kernel + bwd_dq)",
              "decode": "hd_decode_attn (decode_split + decode_combine)",
-             "expand": "hd_expand_embed (expand_kernel)"}[dom["kind"]]
+             "expand": "hd_expand_embed (expand_kernel)",
+             "rope": "hd_rope_expanded (rope_kernel)"}[dom["kind"]]
     roof = {"kernel": f"{kname}, op {dom['name']}", **roof,
             "traffic": NCU_TRAFFIC.get((args.workload, dom["name"]))}
     if hbm_only:

@@ -8,8 +8,9 @@
  *     0-based throughout this library: p = t*n + s, token(p) = p / n,
  *     stream(p) = p % n.
  *   - step 2: the expanded sequence runs through the unchanged Transformer with
- *     causal attention and continuous positions (position encoding is applied
- *     by the caller at the physical position p).
+ *     causal attention and continuous positions: the position encoding runs
+ *     over the physical position p (hd_rope_expanded applies rotary encoding
+ *     there).
  *   - section "规模化落地的工程优化": Stream-Factorized Attention. Intra-stream
  *     layers see only earlier positions of the same stream; cross-stream layers
  *     keep the base model's full-causal or sliding-window attention over the
@@ -82,6 +83,35 @@ int hd_version(void);
  */
 int hd_expand_embed(const int32_t* ids, const void* tables, void* out, int B, int L, int n,
                     int V, int d, int elem_bytes, void* stream);
+
+/*
+ * hd_rope_expanded - rotary position embedding at the physical positions.
+ * Source: tahou.com page, "隐式序列缩放的技术细节" step 2 (the expanded
+ * sequence keeps continuous position encoding). The page does not name the
+ * encoding; this is the rotary form with rotate-half pairing:
+ *
+ *   w_i = base^(-2i/D),  i = 0 .. D/2-1,  angle = p * w_i
+ *   x[i]       <- x[i] cos(angle) - x[i + D/2] sin(angle)
+ *   x[i + D/2] <- x[i + D/2] cos(angle) + x[i] sin(angle)
+ *
+ * applied IN PLACE to every head of the rows of q and k, where p is the
+ * row's physical position: with t0 = token_offset[b] (0 if token_offset is
+ * NULL), row r of k (and of q) is at p = t0*n + r; with
+ * final_stream_queries_only, q row t is at p = (t0 + t)*n + n-1.
+ *
+ *   q            bf16 [B, S, Hq, D] (S = n*L), or [B, L, Hq, D] with
+ *                final_stream_queries_only; NULL skips q
+ *   k            bf16 [B, S, Hkv, D]; NULL skips k (not both NULL)
+ *   token_offset int32 [B] on the device, or NULL: tokens of sequence b that
+ *                precede this call (a decode step passes L = 1 and the
+ *                cached token count). A negative entry leaves that
+ *                sequence's rows unchanged and records HD_ERR_DEVICE_INDEX.
+ *   base         > 1 (10000 in most models)
+ * Supported: D in {16, 32, 64, 128, 256}. The angle is formed and reduced in
+ * fp64, its sine and cosine taken in fp32; the product is rounded to bf16.
+ */
+int hd_rope_expanded(void* q, void* k, const int32_t* token_offset, int B, int L, int n, int Hq,
+                     int Hkv, int D, int final_stream_queries_only, double base, void* stream);
 
 /*
  * hd_attn_fwd - Stream-Factorized attention forward.

@@ -6,6 +6,8 @@ data-parallel hot path of Hidden Decoding with Stream-Factorized Attention
 
 * ``hd_expand_embed``  interleaved n-table embedding gather (stream k of token i
   at position (i-1)n+k);
+* ``hd_rope_expanded``  rotary position embedding of q and k at the physical
+  positions p = t*n + s (continuous positions over the expanded sequence);
 * ``hd_attn_fwd`` / ``hd_attn_bwd``  attention over the expanded sequence with
   intra-stream, cross-stream full-causal and cross-stream sliding-window masks,
   optionally with final-stream-only queries (KV-mirror);
@@ -13,7 +15,7 @@ data-parallel hot path of Hidden Decoding with Stream-Factorized Attention
   interleaved per-stream KV cache.
 
 The C names are re-exported from ``_lib`` (pointer + size arguments). The
-tensor helpers below (``expand_embed``, ``attn_fwd``, ``attn_bwd``,
+tensor helpers below (``expand_embed``, ``rope_``, ``attn_fwd``, ``attn_bwd``,
 ``decode_attn``) allocate outputs and workspace with torch and call the same C
 entry points; torch is used for device memory and streams only.
 """
@@ -35,6 +37,7 @@ from ._lib import (  # noqa: F401
     hd_decode_workspace_bytes,
     hd_device_status,
     hd_expand_embed,
+    hd_rope_expanded,
     lib,
     status_string,
 )
@@ -60,6 +63,26 @@ def expand_embed(ids, tables, stream=None):
     out = torch.empty((B, L * n, d), dtype=tables.dtype, device=tables.device)
     hd_expand_embed(ids, tables, out, B, L, n, V, d, tables.element_size(), stream)
     return out
+
+
+def rope_(q, k, n, final_only=False, base=10000.0, token_offset=None, stream=None):
+    """Rotate q [B, Sq, Hq, D] and k [B, n*L, Hkv, D] bf16 in place at their physical positions.
+
+    Either may be None. ``token_offset`` (int32 [B] on the device) gives the
+    tokens that precede the rows of each sequence. Returns (q, k).
+    """
+    ts = [t for t in (q, k, token_offset) if t is not None]
+    _need_cuda(*ts)
+    ref = k if k is not None else q
+    B, D = ref.shape[0], ref.shape[-1]
+    if k is not None:
+        L = k.shape[1] // n
+    else:
+        L = q.shape[1] if final_only else q.shape[1] // n
+    Hq = q.shape[2] if q is not None else 0
+    Hkv = k.shape[2] if k is not None else 0
+    hd_rope_expanded(q, k, token_offset, B, L, n, Hq, Hkv, D, final_only, base, stream)
+    return q, k
 
 
 def attn_fwd(q, k, v, n, mode, W=0, final_only=False, scale=None, stream=None):

@@ -25,10 +25,12 @@ _P = ctypes.c_void_p
 _I = ctypes.c_int
 _F = ctypes.c_float
 _Z = ctypes.c_size_t
+_D = ctypes.c_double
 SIGNATURES = {
     "hd_status_string": (ctypes.c_char_p, [_I]),
     "hd_version": (_I, []),
     "hd_expand_embed": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
+    "hd_rope_expanded": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _D, _P]),
     "hd_attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "hd_attn_bwd_workspace_bytes": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
     "hd_attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I,
@@ -98,6 +100,12 @@ def _check(st: int, what: str) -> int:
 def hd_expand_embed(ids, tables, out, B, L, n, V, d, elem_bytes, stream=None):
     return _check(lib().hd_expand_embed(ptr(ids), ptr(tables), ptr(out), B, L, n, V, d, elem_bytes,
                                         stream_handle(stream)), "hd_expand_embed")
+
+
+def hd_rope_expanded(q, k, token_offset, B, L, n, Hq, Hkv, D, final_only, base, stream=None):
+    return _check(lib().hd_rope_expanded(ptr(q), ptr(k), ptr(token_offset), B, L, n, Hq, Hkv, D,
+                                         int(final_only), float(base), stream_handle(stream)),
+                  "hd_rope_expanded")
 
 
 def hd_attn_fwd(q, k, v, out, lse, B, L, n, Hq, Hkv, D, mode, W_tokens, final_only, scale,

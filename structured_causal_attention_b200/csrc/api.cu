@@ -2,6 +2,8 @@
 // set-up, launches. Everything is enqueued on the caller's stream; nothing is
 // allocated.
 #include <math.h>
+
+#include <cmath>
 #include <mutex>
 
 #include "hd_common.cuh"
@@ -148,6 +150,33 @@ int hd_expand_embed(const int32_t* ids, const void* tables, void* out, int B, in
     return HD_ERR_INVALID_ARG;
   return from_cuda(launch_expand(ids, tables, out, B, L, n, V, row_bytes, status_ptr(),
                                  static_cast<cudaStream_t>(stream)));
+}
+
+int hd_rope_expanded(void* q, void* k, const int32_t* token_offset, int B, int L, int n, int Hq,
+                     int Hkv, int D, int final_stream_queries_only, double base, void* stream) {
+  if (!q && !k) return HD_ERR_INVALID_ARG;
+  if (B < 1 || L < 1 || n < 1 || D < 1) return HD_ERR_INVALID_ARG;
+  if ((q && Hq < 1) || (k && Hkv < 1)) return HD_ERR_INVALID_ARG;
+  if (final_stream_queries_only != 0 && final_stream_queries_only != 1) return HD_ERR_INVALID_ARG;
+  if (!(base > 1.0) || !std::isfinite(base)) return HD_ERR_INVALID_ARG;
+  if ((q && !aligned16(q)) || (k && !aligned16(k))) return HD_ERR_INVALID_ARG;
+  if (D != 16 && D != 32 && D != 64 && D != 128 && D != 256) return HD_ERR_UNSUPPORTED;
+  if (static_cast<long long>(n) * L > (1LL << 30)) return HD_ERR_UNSUPPORTED;
+  RopeParams p{};
+  p.q = static_cast<__nv_bfloat16*>(q);
+  p.k = static_cast<__nv_bfloat16*>(k);
+  p.token_offset = token_offset;
+  p.status = status_ptr();
+  p.B = B;
+  p.S = n * L;
+  p.Sq = final_stream_queries_only ? L : n * L;
+  p.n = n;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.D = D;
+  p.final_only = final_stream_queries_only;
+  p.log2_base = std::log2(base);
+  return from_cuda(launch_rope(p, static_cast<cudaStream_t>(stream)));
 }
 
 int hd_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int L,

@@ -34,6 +34,16 @@ struct DecodeParams {
 void decode_split_plan(int B, int n, int Tcap, int Hq, int Hkv, int* mt, int* splits, int* chunk);
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
 
+struct RopeParams {
+  __nv_bfloat16* q;             // [B, Sq, Hq, D] or null
+  __nv_bfloat16* k;             // [B, S, Hkv, D] or null
+  const int32_t* token_offset;  // [B] tokens before the call, or null (all 0)
+  int* status;
+  int B, S, Sq, n, Hq, Hkv, D, final_only;
+  double log2_base;
+};
+cudaError_t launch_rope(const RopeParams& p, cudaStream_t stream);
+
 cudaError_t launch_expand(const int32_t* ids, const void* tables, void* out, int B, int L, int n,
                           int V, long long row_bytes, int* status, cudaStream_t stream);
 

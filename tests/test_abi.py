@@ -108,6 +108,25 @@ def test_expand_rejects(lib):
     assert L.hd_expand_embed(FAKE, FAKE + 1, FAKE, 1, 4, 2, 9, 8, 4, None) == hd.HD_ERR_INVALID_ARG
 
 
+def test_rope_rejects(lib):
+    L = hd.lib()
+    ok = [FAKE, FAKE, 0, 2, 8, 4, 8, 2, 128, 0, 10000.0, None]
+    def call(**kw):
+        a = list(ok)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return L.hd_rope_expanded(*a)
+    assert call(a0=0, a1=0) == hd.HD_ERR_INVALID_ARG       # nothing to rotate
+    assert call(a3=0) == hd.HD_ERR_INVALID_ARG             # B
+    assert call(a6=0) == hd.HD_ERR_INVALID_ARG             # Hq with q given
+    assert call(a9=2) == hd.HD_ERR_INVALID_ARG             # final flag
+    assert call(a10=1.0) == hd.HD_ERR_INVALID_ARG          # base must exceed 1
+    assert call(a10=float("inf")) == hd.HD_ERR_INVALID_ARG
+    assert call(a0=FAKE + 8) == hd.HD_ERR_INVALID_ARG      # misaligned
+    assert call(a8=96) == hd.HD_ERR_UNSUPPORTED
+    assert call(a8=512) == hd.HD_ERR_UNSUPPORTED
+
+
 def test_python_binding_raises_on_error(lib):
     with pytest.raises(hd.HDError) as e:
         hd.hd_attn_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 4, 4, 2, 96, 0, 1, 0, 0.1, stream=0)

@@ -74,8 +74,8 @@ MUTANTS = [
      [(pins.test_n1_reduces_to_textbook_causal, "CROSS_FULL")]),
     ("stream-major expansion", oracle.expand, "out[:, s::n, :] = tables[s][ids]",
      "out[:, s * L:(s + 1) * L, :] = tables[s][ids]", [(pins.test_golden_expand, "G")]),
-    ("decode query at stream 0", oracle.decode, "qpos = T * n + np.arange(n)",
-     "qpos = T * n + 0 * np.arange(n)",
+    ("decode query at stream 0", oracle.decode, "qpos = T * n + streams",
+     "qpos = T * n + 0 * streams",
      [(pins.test_golden_decode, "G")]),
 ]
 

@@ -393,6 +393,47 @@ def test_decode_equals_prefill_rows(name):
         np.testing.assert_allclose(lse[b], fl[0, :, Tb * n:], atol=1e-12)
 
 
+@pytest.mark.parametrize("name", list(MODES))
+def test_final_only_decode_equals_final_only_prefill_last_row(name):
+    """One query per sequence at T*n + n-1 = the last row of a final-stream-only prefill."""
+    n, Tcap, Hq, Hkv, D, W = 4, 7, 6, 3, 8, 2
+    mode = MODES[name]
+    B = 3
+    kc, vc = _rand((B, Tcap * n, Hkv, D), 46), _rand((B, Tcap * n, Hkv, D), 47)
+    q = _rand((B, 1, Hq, D), 48)
+    seqlen = np.array([Tcap, 1, 3])
+    o, lse = oracle.decode_attn(q, kc, vc, seqlen, n, mode, W, 0.4, final_only=True)
+    assert o.shape == (B, 1, Hq, D) and lse.shape == (B, Hq, 1)
+    for b in range(B):
+        T1 = int(seqlen[b])
+        qf = np.zeros((1, T1, Hq, D))
+        qf[0, T1 - 1] = q[b, 0]
+        fo, fl = oracle.attn_fwd(qf, kc[b:b + 1, :T1 * n], vc[b:b + 1, :T1 * n], n, mode, W, True, 0.4)
+        np.testing.assert_allclose(o[b, 0], fo[0, T1 - 1], atol=1e-12)
+        np.testing.assert_allclose(lse[b, :, 0], fl[0, :, T1 - 1], atol=1e-12)
+
+
+def test_final_only_intra_decode_reads_only_the_final_stream():
+    """INTRA, final stream: the other streams' cache rows do not change the result."""
+    n, Tcap, Hq, Hkv, D = 3, 5, 2, 1, 8
+    kc, vc = _rand((1, Tcap * n, Hkv, D), 49), _rand((1, Tcap * n, Hkv, D), 50)
+    q = _rand((1, 1, Hq, D), 51)
+    o1, l1 = oracle.decode_attn(q, kc, vc, [Tcap], n, MODES["INTRA"], 1, 0.5, final_only=True)
+    kc2, vc2 = kc.copy(), vc.copy()
+    other = np.arange(Tcap * n) % n != n - 1
+    kc2[:, other] = 7.0
+    vc2[:, other] = -3.0
+    o2, l2 = oracle.decode_attn(q, kc2, vc2, [Tcap], n, MODES["INTRA"], 1, 0.5, final_only=True)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+    # and equals plain softmax attention over the final stream's rows
+    kk, vv = kc[0, n - 1::n, 0], vc[0, n - 1::n, 0]
+    for h in range(Hq):
+        sc = 0.5 * kk @ q[0, 0, h]
+        w = np.exp(sc - sc.max())
+        np.testing.assert_allclose(o1[0, 0, h], (w / w.sum()) @ vv, atol=1e-12)
+
+
 # ---------------------------------------------------------------- expansion
 
 @pytest.mark.parametrize("B,L,n,V,d", [(1, 5, 3, 7, 4), (2, 3, 1, 5, 6), (3, 4, 4, 9, 1)])

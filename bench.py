@@ -85,6 +85,14 @@ def step_plan(wl):
         io = B * n * Hq * D * 2 * 2 + B * Hq * n * 4
         ops.append(dict(name=f"decode_{name}", kind="decode", mode=mode, fin=0, flops=4 * D * pr,
                         pairs=pr, bytes=kv_bytes + io))
+    for name, mode in (("cross_full", CROSS_FULL), ("intra", INTRA)):
+        # final stream alone: INTRA reads only that stream's T+1 rows
+        rows = (T + 1) * (n if mode == CROSS_FULL else 1)
+        pr = B * Hq * rows
+        kv_bytes = 2 * B * rows * Hkv * D * 2
+        io = B * Hq * D * 2 * 2 + B * Hq * 4
+        ops.append(dict(name=f"decode_final_{name}", kind="decode_final", mode=mode, fin=1,
+                        flops=4 * D * pr, pairs=pr, bytes=kv_bytes + io))
     ex_bytes = B * L * 4 + 2 * B * L * n * wl["d"] * 4
     ops.insert(0, dict(name="expand", kind="expand", flops=0, pairs=0, bytes=ex_bytes))
     # rotary embedding of q and k in place: every element read and written once
@@ -92,9 +100,9 @@ def step_plan(wl):
     return ops
 
 
-LAUNCHES = {"expand": 1, "fwd": 1, "bwd": 3, "decode": 2, "rope": 1}
+LAUNCHES = {"expand": 1, "fwd": 1, "bwd": 3, "decode": 2, "decode_final": 2, "rope": 1}
 # operations measured on their own only (not part of the default hot-path step)
-EXTRA_KINDS = {"rope"}
+EXTRA_KINDS = {"rope", "decode_final"}
 
 # Extra workloads for per-configuration measurements (`--workload`); the
 # default is the whole hot-path step above.
@@ -112,6 +120,8 @@ WORKLOADS = {
                      ops=["decode_cross_full", "decode_intra"]),
     "expand": dict(B=4, L=8192, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=1,
                    ops=["expand"]),
+    "decode8_final": dict(B=8, L=1, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=16384,
+                          ops=["decode_final_cross_full", "decode_final_intra"]),
     "rope": dict(B=1, L=32768, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=1,
                  ops=["rope"]),
 }
@@ -163,6 +173,8 @@ class Step:
                     self.h["dof"] = syn.normal_bf16((B, L, Hq, D), 13)
         if "decode" in kinds:
             self.h["dq_new"] = syn.normal_bf16((B, n, Hq, D), 14)
+        if "decode_final" in kinds:
+            self.h["dq_fin"] = syn.normal_bf16((B, 1, Hq, D), 18)
         if "rope" in kinds and not attn:
             self.h["q"] = syn.normal_bf16((B, S, Hq, D), 16)
             self.h["k"] = syn.normal_bf16((B, S, Hkv, D), 17)
@@ -175,14 +187,21 @@ class Step:
         if "expand" in kinds:
             self.tables = torch.empty((n, V, d), dtype=torch.float32, device=dev).normal_(0, 0.02, generator=g)
             self.x = torch.empty((B, S, d), dtype=torch.float32, device=dev)
-        if "decode" in kinds:
+        if kinds & {"decode", "decode_final"}:
             self.kc = torch.empty((B, (T + 1) * n, Hkv, D), dtype=torch.bfloat16, device=dev).normal_(generator=g)
             self.vc = torch.empty_like(self.kc).normal_(generator=g)
             self.seqlen = torch.full((B,), T + 1, dtype=torch.int32, device=dev)
+        if "decode" in kinds:
             self.ws_dec_n = hd.hd_decode_workspace_bytes(B, n, T + 1, Hq, Hkv, D)
             self.ws_dec = torch.empty(self.ws_dec_n, dtype=torch.uint8, device=dev)
             self.dec_o = {m: torch.empty_like(self.d["dq_new"]) for m in ("cross_full", "intra")}
             self.dec_l = {m: torch.empty((B, Hq, n), dtype=torch.float32, device=dev)
+                          for m in ("cross_full", "intra")}
+        if "decode_final" in kinds:
+            self.ws_fin_n = hd.hd_decode_final_workspace_bytes(B, n, T + 1, Hq, Hkv, D)
+            self.ws_fin = torch.empty(self.ws_fin_n, dtype=torch.uint8, device=dev)
+            self.fin_o = {m: torch.empty_like(self.d["dq_fin"]) for m in ("cross_full", "intra")}
+            self.fin_l = {m: torch.empty((B, Hq, 1), dtype=torch.float32, device=dev)
                           for m in ("cross_full", "intra")}
         self.o, self.lse = {}, {}
         for o in ops:
@@ -206,6 +225,8 @@ class Step:
         self.result = []
         if "decode" in kinds:
             self.result += list(self.dec_o.values())
+        elif "decode_final" in kinds:
+            self.result += list(self.fin_o.values())
         elif self.lse:
             self.result.append(next(iter(self.lse.values())))
         elif "expand" in kinds:
@@ -237,6 +258,11 @@ class Step:
                 hd.hd_attn_bwd(q, d["k"], d["v"], self.o[key], self.lse[key], do,
                                self.dqf if fin else self.dq, self.dk, self.dv, B, L, n, Hq, Hkv, D,
                                op["mode"], W, fin, sc, self.ws_bwd, self.ws_bwd_n, s)
+        elif op["kind"] == "decode_final":
+            key = name.split("_", 2)[2]
+            hd.hd_decode_attn_final(d["dq_fin"], self.kc, self.vc, self.seqlen, self.fin_o[key],
+                                    self.fin_l[key], B, n, T + 1, Hq, Hkv, D, op["mode"], W, sc,
+                                    self.ws_fin, self.ws_fin_n, s)
         else:
             key = name.split("_", 1)[1]
             hd.hd_decode_attn(d["dq_new"], self.kc, self.vc, self.seqlen, self.dec_o[key],
@@ -384,6 +410,8 @@ DESCRIPTIONS = {
     "decode8": "decode step CROSS_FULL + INTRA, B8 n4, 16384 prior tokens (65540 cache rows), Hq32 Hkv8 D128",
     "decode64": "decode step CROSS_FULL + INTRA, B64 n4, 16384 prior tokens (65540 cache rows), Hq32 Hkv8 D128",
     "expand": "expansion B4 L8192 n4, V32000, d4096 fp32 tables",
+    "decode8_final": "final-stream-only decode (one query per sequence) CROSS_FULL + INTRA, B8 n4, "
+                     "16384 prior tokens (65540 cache rows), Hq32 Hkv8 D128",
     "rope": "RoPE in place at physical positions, q [1,131072,32,128] + k [1,131072,8,128] bf16, base 10000",
 }
 
@@ -409,7 +437,7 @@ def main():
     wl, ops = plan_for(args.workload)
     total_flops = sum(o["flops"] for o in ops)
     total_bytes = sum(o.get("bytes", 0) for o in ops)
-    hbm_only = total_flops == 0 or all(o["kind"] in ("decode", "expand", "rope") for o in ops)
+    hbm_only = total_flops == 0 or all(o["kind"] in ("decode", "decode_final", "expand", "rope") for o in ops)
     tokens = wl["B"] * wl["n"] * wl["L"]
     config = {"workload": DESCRIPTIONS[args.workload],
               "global_batch": wl["B"] * max(world, 1), "seq_len": wl["n"] * wl["L"],
@@ -559,6 +587,7 @@ def main():
              "bwd": "hd_attn_bwd (bwd_pre + attn_bwd_tc_kernel + bwd_dq)",
              "decode": "hd_decode_attn (decode_split + decode_combine)",
              "expand": "hd_expand_embed (expand_kernel)",
+             "decode_final": "hd_decode_attn_final (decode_split + decode_combine)",
              "rope": "hd_rope_expanded (rope_kernel)"}[dom["kind"]]
     roof = {"kernel": f"{kname}, op {dom['name']}", **roof,
             "traffic": NCU_TRAFFIC.get((args.workload, dom["name"]))}

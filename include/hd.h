@@ -182,6 +182,30 @@ int hd_decode_attn(const void* q, const void* k_cache, const void* v_cache, cons
                    int W_tokens, float scale, void* workspace, size_t workspace_bytes,
                    void* stream);
 
+/* Bytes of workspace hd_decode_attn_final needs for these sizes, whatever the
+ * mode (0 on invalid sizes). */
+size_t hd_decode_final_workspace_bytes(int B, int n, int Tcap, int Hq, int Hkv, int D);
+
+/*
+ * hd_decode_attn_final - final-stream-only decode (KV-mirror layers).
+ * Source: tahou.com page, "规模化落地的工程优化", KV-mirror paragraph (only the
+ * last stream passes through the mirror layers, which read K/V built for all
+ * streams).
+ *
+ * As hd_decode_attn, with one query per sequence: stream n-1 of the new
+ * token, at p = T*n + n-1.
+ *   q    bf16 [B, 1, Hq, D] (equivalently [B, Hq, D])
+ *   out  bf16 [B, 1, Hq, D]; lse fp32 [B, Hq] (= [B, Hq, 1])
+ *   k_cache, v_cache, seqlen, mode, W_tokens, scale: as hd_decode_attn
+ *        (same precondition: the new token's n K/V rows are in the cache).
+ * Under HD_INTRA only the final stream's cache rows (positions n-1, 2n-1, ...)
+ * are read. `workspace` must hold hd_decode_final_workspace_bytes(...) bytes.
+ */
+int hd_decode_attn_final(const void* q, const void* k_cache, const void* v_cache,
+                         const int32_t* seqlen, void* out, float* lse, int B, int n, int Tcap,
+                         int Hq, int Hkv, int D, int mode, int W_tokens, float scale,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
 /*
  * hd_decode_attn_noalloc - hd_decode_attn for callers that cannot allocate.
  * The pages have no counterpart: this is a deployment convenience.

@@ -11,12 +11,13 @@ data-parallel hot path of Hidden Decoding with Stream-Factorized Attention
 * ``hd_attn_fwd`` / ``hd_attn_bwd``  attention over the expanded sequence with
   intra-stream, cross-stream full-causal and cross-stream sliding-window masks,
   optionally with final-stream-only queries (KV-mirror);
+* ``hd_decode_attn_final``  the final stream's query alone (KV-mirror layers);
 * ``hd_decode_attn``  the n stream queries of a new token against the
   interleaved per-stream KV cache.
 
 The C names are re-exported from ``_lib`` (pointer + size arguments). The
 tensor helpers below (``expand_embed``, ``rope_``, ``attn_fwd``, ``attn_bwd``,
-``decode_attn``) allocate outputs and workspace with torch and call the same C
+``decode_attn``, ``decode_attn_final``) allocate outputs and workspace with torch and call the same C
 entry points; torch is used for device memory and streams only.
 """
 from __future__ import annotations
@@ -33,7 +34,9 @@ from ._lib import (  # noqa: F401
     hd_attn_bwd_workspace_bytes,
     hd_attn_fwd,
     hd_decode_attn,
+    hd_decode_attn_final,
     hd_decode_attn_noalloc,
+    hd_decode_final_workspace_bytes,
     hd_decode_workspace_bytes,
     hd_device_status,
     hd_expand_embed,
@@ -138,4 +141,30 @@ def decode_attn(q, k_cache, v_cache, seqlen, mode, W=0, scale=None, stream=None,
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
     hd_decode_attn(q, k_cache, v_cache, seqlen, out, lse, B, n, Tcap, Hq, Hkv, D, mode, W, scale,
                    workspace, workspace.numel() * workspace.element_size(), stream)
+    return out, lse
+
+
+def decode_attn_final(q, k_cache, v_cache, seqlen, n, mode, W=0, scale=None, stream=None,
+                      workspace=None):
+    """q [B, 1, Hq, D] (stream n-1 of the new token); caches [B, Tcap*n, Hkv, D]; seqlen int32 [B].
+
+    Returns (out [B, 1, Hq, D] bf16, lse [B, Hq, 1] fp32).
+    """
+    import torch
+
+    _need_cuda(q, k_cache, v_cache, seqlen)
+    B, one, Hq, D = q.shape
+    if one != 1:
+        raise ValueError("q must be [B, 1, Hq, D]")
+    Hkv = k_cache.shape[2]
+    Tcap = k_cache.shape[1] // n
+    if scale is None:
+        scale = D ** -0.5
+    out = torch.empty_like(q)
+    lse = torch.empty((B, Hq, 1), dtype=torch.float32, device=q.device)
+    nbytes = hd_decode_final_workspace_bytes(B, n, Tcap, Hq, Hkv, D)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    hd_decode_attn_final(q, k_cache, v_cache, seqlen, out, lse, B, n, Tcap, Hq, Hkv, D, mode, W,
+                         scale, workspace, workspace.numel() * workspace.element_size(), stream)
     return out, lse

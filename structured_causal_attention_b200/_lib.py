@@ -38,6 +38,9 @@ SIGNATURES = {
     "hd_decode_workspace_bytes": (_Z, [_I, _I, _I, _I, _I, _I]),
     "hd_decode_attn": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _Z,
                             _P]),
+    "hd_decode_final_workspace_bytes": (_Z, [_I, _I, _I, _I, _I, _I]),
+    "hd_decode_attn_final": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P,
+                                  _Z, _P]),
     "hd_decode_attn_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F,
                                     _P]),
     "hd_device_status": (_I, [_P, _I]),
@@ -137,6 +140,19 @@ def hd_decode_attn(q, k_cache, v_cache, seqlen, out, lse, B, n, Tcap, Hq, Hkv, D
                                        ptr(lse), B, n, Tcap, Hq, Hkv, D, mode, W_tokens, float(scale),
                                        ptr(workspace), int(workspace_bytes), stream_handle(stream)),
                   "hd_decode_attn")
+
+
+def hd_decode_final_workspace_bytes(B, n, Tcap, Hq, Hkv, D):
+    return int(lib().hd_decode_final_workspace_bytes(B, n, Tcap, Hq, Hkv, D))
+
+
+def hd_decode_attn_final(q, k_cache, v_cache, seqlen, out, lse, B, n, Tcap, Hq, Hkv, D, mode,
+                         W_tokens, scale, workspace, workspace_bytes, stream=None):
+    return _check(lib().hd_decode_attn_final(ptr(q), ptr(k_cache), ptr(v_cache), ptr(seqlen),
+                                             ptr(out), ptr(lse), B, n, Tcap, Hq, Hkv, D, mode,
+                                             W_tokens, scale, ptr(workspace), workspace_bytes,
+                                             stream_handle(stream)),
+                  "hd_decode_attn_final")
 
 
 def hd_decode_attn_noalloc(q, k_cache, v_cache, seqlen, out, lse, B, n, Tcap, Hq, Hkv, D, mode,

@@ -117,6 +117,87 @@ size_t packed_rows(int B, int L, int n, int Hq, int final_only) {
 
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? HD_OK : HD_ERR_CUDA; }
 
+// Split-K partials for `rows` query rows per (sequence, KV head) against up to
+// `keys` keys: unnormalised O (fp32 [.., D]) and (max, sum) pairs.
+size_t decode_partials_bytes(int B, int rows, long long keys, int Hkv, int D) {
+  int mt = 0, splits = 0, chunk = 0;
+  decode_split_plan(B, rows, keys, Hkv, &mt, &splits, &chunk);
+  const size_t prow = static_cast<size_t>(B) * Hkv * mt * 16 * splits;
+  return align256(prow * static_cast<size_t>(D) * 4) + align256(prow * 2 * 4);
+}
+
+// Workspace of one decode call. All n streams: n*g rows over the whole cache.
+// Final stream alone: g rows over the whole cache (CROSS modes) or over its
+// own Tcap rows (INTRA); the workspace covers both, so it does not depend on
+// the mode.
+size_t decode_workspace(int B, int n, int Tcap, int Hq, int Hkv, int D, int final_only) {
+  if (B < 1 || n < 1 || Tcap < 1 || Hq < 1 || Hkv < 1 || D < 1 || Hq % Hkv) return 0;
+  const int g = Hq / Hkv;
+  const long long keys = static_cast<long long>(Tcap) * n;
+  if (!final_only) return decode_partials_bytes(B, n * g, keys, Hkv, D);
+  const size_t a = decode_partials_bytes(B, g, keys, Hkv, D);
+  const size_t b = decode_partials_bytes(B, g, Tcap, Hkv, D);
+  return a > b ? a : b;
+}
+
+int decode_call(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlen,
+                void* out, float* lse, int B, int n, int Tcap, int Hq, int Hkv, int D, int mode,
+                int W_tokens, int final_only, float scale, void* workspace,
+                size_t workspace_bytes, void* stream) {
+  if (!q || !k_cache || !v_cache || !seqlen || !out || !lse || !workspace) return HD_ERR_INVALID_ARG;
+  if (B < 1 || n < 1 || Tcap < 1 || Hq < 1 || Hkv < 1 || D < 1) return HD_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return HD_ERR_INVALID_ARG;
+  if (mode < HD_INTRA || mode > HD_CROSS_WINDOW) return HD_ERR_INVALID_ARG;
+  if (mode == HD_CROSS_WINDOW && W_tokens < 1) return HD_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return HD_ERR_INVALID_ARG;
+  if (static_cast<long long>(Tcap) * n > kMaxPositions) return HD_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return HD_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+      !aligned16(workspace))
+    return HD_ERR_INVALID_ARG;
+  const size_t need = decode_workspace(B, n, Tcap, Hq, Hkv, D, final_only);
+  if (workspace_bytes < need) return HD_ERR_INVALID_ARG;
+  DecodeParams p = {};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.kc = static_cast<const __nv_bfloat16*>(k_cache);
+  p.vc = static_cast<const __nv_bfloat16*>(v_cache);
+  p.seqlen = seqlen;
+  p.o = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.status = status_ptr();
+  p.B = B;
+  p.n = n;
+  p.Tcap = Tcap;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.D = D;
+  p.mode = mode;
+  const long long w = static_cast<long long>(n) * W_tokens;
+  p.win = (mode == HD_CROSS_WINDOW && w < static_cast<long long>(Tcap) * n) ? static_cast<int>(w)
+                                                                           : kWinInf;
+  if (mode == HD_CROSS_WINDOW && p.win == kWinInf) p.mode = HD_CROSS_FULL;
+  p.nq = final_only ? 1 : n;
+  p.s0 = final_only ? n - 1 : 0;
+  p.kstride = 1;
+  p.kres = 0;
+  p.kpt = n;
+  if (final_only && mode == HD_INTRA && n > 1) {
+    // the final stream's own rows only; each of them is visible to its query
+    p.kstride = n;
+    p.kres = n - 1;
+    p.kpt = 1;
+    p.mode = HD_CROSS_FULL;
+  }
+  p.rows = p.nq * (Hq / Hkv);
+  decode_split_plan(B, p.rows, static_cast<long long>(Tcap) * p.kpt, Hkv, &p.mt, &p.splits,
+                    &p.chunk);
+  const size_t prow = static_cast<size_t>(B) * Hkv * p.mt * 16 * p.splits;
+  p.part_o = static_cast<float*>(workspace);
+  p.part_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(prow * D * 4));
+  p.scale_log2 = scale * 1.4426950408889634074f;
+  return from_cuda(launch_decode(p, static_cast<cudaStream_t>(stream)));
+}
+
 }  // namespace
 }  // namespace hd
 
@@ -231,56 +312,27 @@ int hd_attn_bwd(const void* q, const void* k, const void* v, const void* out, co
 }
 
 size_t hd_decode_workspace_bytes(int B, int n, int Tcap, int Hq, int Hkv, int D) {
-  if (B < 1 || n < 1 || Tcap < 1 || Hq < 1 || Hkv < 1 || D < 1 || Hq % Hkv) return 0;
-  int mt = 0, splits = 0, chunk = 0;
-  decode_split_plan(B, n, Tcap, Hq, Hkv, &mt, &splits, &chunk);
-  const size_t prow = static_cast<size_t>(B) * Hkv * mt * 16 * splits;
-  return align256(prow * static_cast<size_t>(D) * 4) + align256(prow * 2 * 4);
+  return hd::decode_workspace(B, n, Tcap, Hq, Hkv, D, 0);
+}
+
+size_t hd_decode_final_workspace_bytes(int B, int n, int Tcap, int Hq, int Hkv, int D) {
+  return hd::decode_workspace(B, n, Tcap, Hq, Hkv, D, 1);
 }
 
 int hd_decode_attn(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlen,
                    void* out, float* lse, int B, int n, int Tcap, int Hq, int Hkv, int D, int mode,
                    int W_tokens, float scale, void* workspace, size_t workspace_bytes,
                    void* stream) {
-  if (!q || !k_cache || !v_cache || !seqlen || !out || !lse || !workspace) return HD_ERR_INVALID_ARG;
-  if (B < 1 || n < 1 || Tcap < 1 || Hq < 1 || Hkv < 1 || D < 1) return HD_ERR_INVALID_ARG;
-  if (Hq % Hkv != 0) return HD_ERR_INVALID_ARG;
-  if (mode < HD_INTRA || mode > HD_CROSS_WINDOW) return HD_ERR_INVALID_ARG;
-  if (mode == HD_CROSS_WINDOW && W_tokens < 1) return HD_ERR_INVALID_ARG;
-  if (!(scale > 0.f) || !isfinite(scale)) return HD_ERR_INVALID_ARG;
-  if (static_cast<long long>(Tcap) * n > kMaxPositions) return HD_ERR_UNSUPPORTED;
-  if (D != 64 && D != 128) return HD_ERR_UNSUPPORTED;
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
-      !aligned16(workspace))
-    return HD_ERR_INVALID_ARG;
-  const size_t need = hd_decode_workspace_bytes(B, n, Tcap, Hq, Hkv, D);
-  if (workspace_bytes < need) return HD_ERR_INVALID_ARG;
-  DecodeParams p = {};
-  p.q = static_cast<const __nv_bfloat16*>(q);
-  p.kc = static_cast<const __nv_bfloat16*>(k_cache);
-  p.vc = static_cast<const __nv_bfloat16*>(v_cache);
-  p.seqlen = seqlen;
-  p.o = static_cast<__nv_bfloat16*>(out);
-  p.lse = lse;
-  p.status = status_ptr();
-  p.B = B;
-  p.n = n;
-  p.Tcap = Tcap;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.D = D;
-  p.mode = mode;
-  const long long w = static_cast<long long>(n) * W_tokens;
-  p.win = (mode == HD_CROSS_WINDOW && w < static_cast<long long>(Tcap) * n) ? static_cast<int>(w)
-                                                                           : kWinInf;
-  if (mode == HD_CROSS_WINDOW && p.win == kWinInf) p.mode = HD_CROSS_FULL;
-  p.rows = n * (Hq / Hkv);
-  decode_split_plan(B, n, Tcap, Hq, Hkv, &p.mt, &p.splits, &p.chunk);
-  const size_t prow = static_cast<size_t>(B) * Hkv * p.mt * 16 * p.splits;
-  p.part_o = static_cast<float*>(workspace);
-  p.part_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(prow * D * 4));
-  p.scale_log2 = scale * 1.4426950408889634074f;
-  return from_cuda(launch_decode(p, static_cast<cudaStream_t>(stream)));
+  return hd::decode_call(q, k_cache, v_cache, seqlen, out, lse, B, n, Tcap, Hq, Hkv, D, mode,
+                         W_tokens, 0, scale, workspace, workspace_bytes, stream);
+}
+
+int hd_decode_attn_final(const void* q, const void* k_cache, const void* v_cache,
+                         const int32_t* seqlen, void* out, float* lse, int B, int n, int Tcap,
+                         int Hq, int Hkv, int D, int mode, int W_tokens, float scale,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  return hd::decode_call(q, k_cache, v_cache, seqlen, out, lse, B, n, Tcap, Hq, Hkv, D, mode,
+                         W_tokens, 1, scale, workspace, workspace_bytes, stream);
 }
 
 int hd_device_status(void* stream, int clear) {

@@ -7,6 +7,10 @@
 //
 // Query s of sequence b sits at p = T*n + s (T = seqlen[b]-1) and reads cache
 // positions c with c <= p, plus c % n == s (INTRA) or p - c < n*W (CROSS_WINDOW).
+// Final-stream-only decode (section "规模化落地的工程优化", KV-mirror: only the
+// last stream passes through the mirror layers) runs the query s = n-1 alone;
+// under INTRA it then reads only the final stream's cache rows (every n-th row),
+// for which every loaded key is visible.
 //
 // Split-K: each CTA owns (batch, KV head, 16-row tile of the n*group query
 // rows, key chunk). K/V blocks of 64 positions stream once through a 3-stage
@@ -62,8 +66,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
   const bool ok = seq_ok(T1, p.Tcap);
   if (!ok && tid == 0 && mt == 0 && split == 0 && hk == 0) record_status(p.status, HD_ERR_DEVICE_INDEX);
   const int T = ok ? T1 - 1 : 0;
-  const int kend = ok ? T1 * p.n : 0;
-  const int kbeg = (p.mode == HD_CROSS_WINDOW) ? max(0, T * p.n - p.win + 1) : 0;
+  // key-space range: [kbeg, kend); with kstride 1 key index = cache position
+  const int kend = ok ? T1 * p.kpt : 0;
+  const int kbeg = (p.mode == HD_CROSS_WINDOW) ? max(0, T * p.n + p.s0 - p.win + 1) : 0;
   const int cs = kbeg + split * p.chunk;
   const int ce = min(kend, cs + p.chunk);
   const long long part_row0 = (static_cast<long long>(b) * p.Hkv + hk) * rows_pad + mt * 16;
@@ -77,12 +82,12 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
     return;
   }
 
-  // ---- Q rows of this tile: row i = s*g + j -> q[b, s, hk*g + j, :]
+  // ---- Q rows of this tile: row i = s*g + j -> q[b, s, hk*g + j, :] (s local to the nq streams)
   for (int i = tid; i < 16 * RC; i += kDecThreads) {
     const int lr = i / RC, ch = i % RC, row = mt * 16 + lr;
     const bool valid = row < p.rows;
     const int s = valid ? row / g : 0, j = valid ? row % g : 0;
-    const __nv_bfloat16* src = p.q + ((static_cast<long long>(b) * p.n + s) * p.Hq + hk * g + j) * D + ch * 8;
+    const __nv_bfloat16* src = p.q + ((static_cast<long long>(b) * p.nq + s) * p.Hq + hk * g + j) * D + ch * 8;
     cp_async16(sQ + swz(lr, ch, RC), src, valid ? 16 : 0);
   }
   const long long kv_rs = static_cast<long long>(p.Hkv) * D;
@@ -94,7 +99,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
     const uint32_t dk = sStage + st * SM::STAGE, dv = dk + SM::STAGE / 2;
     for (int i = tid; i < kDecBlk * RC; i += kDecThreads) {
       const int row = i / RC, ch = i % RC, c = base + row;
-      const long long off = static_cast<long long>(min(c, ce - 1)) * kv_rs + ch * 8;
+      const long long pos = p.kres + static_cast<long long>(min(c, ce - 1)) * p.kstride;
+      const long long off = pos * kv_rs + ch * 8;
       const int nb = c < ce ? 16 : 0;
       cp_async16(dk + swz(row, ch, RC), kg + off, nb);
       cp_async16(dv + swz(row, ch, RC), vg + off, nb);
@@ -118,8 +124,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
   for (int hr = 0; hr < 2; ++hr) {
     const int row = mt * 16 + (lane >> 2) + hr * 8;
     rvalid[hr] = row < p.rows;
-    srow[hr] = rvalid[hr] ? row / g : 0;
-    prow[hr] = T * p.n + srow[hr];
+    srow[hr] = p.s0 + (rvalid[hr] ? row / g : 0);
+    // the query's own key index: its position, or (final stream alone) its token
+    prow[hr] = (p.kstride == 1) ? T * p.n + srow[hr] : T;
   }
   // INTRA: key c is visible iff c % n == s. Blocks start at multiples of 64,
   // so c % n = (block base % n + offset % n) mod n: the offsets' residues are
@@ -269,7 +276,7 @@ __global__ void decode_combine_kernel(const DecodeParams p) {
   const int hk = static_cast<int>((gi / p.rows) % p.Hkv);
   const int b = static_cast<int>(gi / (static_cast<long long>(p.rows) * p.Hkv));
   const int g = p.Hq / p.Hkv;
-  const int s = row / g, h = hk * g + row % g;
+  const int s = row / g, h = hk * g + row % g;  // s local to the nq query streams
   const long long prow = (static_cast<long long>(b) * p.Hkv + hk) * (p.mt * 16) + row;
   const bool ok = seq_ok(p.seqlen[b], p.Tcap);
 
@@ -295,11 +302,11 @@ __global__ void decode_combine_kernel(const DecodeParams p) {
     for (int i = 0; i < PER; ++i) acc[i] += f * po[lane + 32 * i];
   }
   const float inv = (ok && lt > 0.f) ? 1.f / lt : 0.f;
-  __nv_bfloat16* out = p.o + ((static_cast<long long>(b) * p.n + s) * p.Hq + h) * D;
+  __nv_bfloat16* out = p.o + ((static_cast<long long>(b) * p.nq + s) * p.Hq + h) * D;
 #pragma unroll
   for (int i = 0; i < PER; ++i) out[lane + 32 * i] = __float2bfloat16_rn(acc[i] * inv);
   if (lane == 0)
-    p.lse[(static_cast<long long>(b) * p.Hq + h) * p.n + s] =
+    p.lse[(static_cast<long long>(b) * p.Hq + h) * p.nq + s] =
         (ok && lt > 0.f) ? (mx + __log2f(lt)) * kLn2 : -INFINITY;
 }
 
@@ -320,11 +327,9 @@ cudaError_t launch_decode_d(const DecodeParams& p, cudaStream_t stream) {
 
 }  // namespace
 
-void decode_split_plan(int B, int n, int Tcap, int Hq, int Hkv, int* mt, int* splits, int* chunk) {
-  const int rows = n * (Hq / Hkv);
+void decode_split_plan(int B, int rows, long long keys, int Hkv, int* mt, int* splits, int* chunk) {
   const int m = (rows + 15) / 16;
   const long long units = static_cast<long long>(B) * Hkv * m;
-  const long long keys = static_cast<long long>(Tcap) * n;
   const long long target = 148LL * 2 * 4;  // 4 waves of 2 resident CTAs per SM
   long long sp = (target + units - 1) / units;
   // at least 8 blocks (512 keys) per split, so that short caches are not cut

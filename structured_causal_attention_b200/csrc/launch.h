@@ -16,22 +16,29 @@ cudaError_t launch_attn_bwd(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_attn_bwd_tc_main(const AttnParams& p, cudaStream_t stream);
 
 struct DecodeParams {
-  const __nv_bfloat16* q;   // [B, n, Hq, D]
+  const __nv_bfloat16* q;   // [B, nq, Hq, D]
   const __nv_bfloat16* kc;  // [B, Tcap*n, Hkv, D]
   const __nv_bfloat16* vc;
   const int32_t* seqlen;    // [B]
-  __nv_bfloat16* o;         // [B, n, Hq, D]
-  float* lse;               // [B, Hq, n]
+  __nv_bfloat16* o;         // [B, nq, Hq, D]
+  float* lse;               // [B, Hq, nq]
   float* part_o;            // [B, Hkv, MT*16, splits, D] fp32
   float* part_ml;           // [B, Hkv, MT*16, splits, 2] fp32 (max in log2 units, sum)
   int* status;
   int B, n, Tcap, Hq, Hkv, D, mode, win;  // win = n*W or kWinInf
-  int rows, mt, splits, chunk;             // rows = n*(Hq/Hkv); chunk keys per split
+  // Query streams s0 .. s0+nq-1 of the new token (all n, or only the final one).
+  int nq, s0;
+  // Keys are indexed in a "key space": key index c is cache position
+  // kres + c*kstride, and a sequence of T1 tokens holds T1*kpt keys. The whole
+  // cache: (1, 0, n). The final stream alone (final-stream-only INTRA): (n, n-1, 1).
+  int kstride, kres, kpt;
+  int rows, mt, splits, chunk;             // rows = nq*(Hq/Hkv); chunk keys per split
   float scale_log2;
 };
 
-// Number of splits / chunk length the decode launcher uses for these sizes.
-void decode_split_plan(int B, int n, int Tcap, int Hq, int Hkv, int* mt, int* splits, int* chunk);
+// Number of splits / chunk length the decode launcher uses for `rows` query
+// rows per (sequence, KV head) against up to `keys` keys.
+void decode_split_plan(int B, int rows, long long keys, int Hkv, int* mt, int* splits, int* chunk);
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
 
 struct RopeParams {

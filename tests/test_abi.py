@@ -100,6 +100,23 @@ def test_decode_rejects(lib):
     assert L.hd_decode_attn(0, *base[1:], *ok, FAKE, ws, None) == hd.HD_ERR_INVALID_ARG
 
 
+def test_decode_final_workspace_and_rejects(lib):
+    L = hd.lib()
+    B, n, Tcap, Hq, Hkv, D = 2, 4, 100, 16, 4, 128
+    ws = hd.hd_decode_final_workspace_bytes(B, n, Tcap, Hq, Hkv, D)
+    assert ws > 0 and hd.hd_decode_final_workspace_bytes(B, n, Tcap, 15, Hkv, D) == 0
+    base = [FAKE] * 6
+    ok = [B, n, Tcap, Hq, Hkv, D, hd.INTRA, 1, 0.1]
+    assert L.hd_decode_attn_final(*base, *ok, FAKE, ws - 1, None) == hd.HD_ERR_INVALID_ARG
+    bad = list(ok)
+    bad[5] = 96
+    assert L.hd_decode_attn_final(*base, *bad, FAKE, ws, None) == hd.HD_ERR_UNSUPPORTED
+    bad = list(ok)
+    bad[6], bad[7] = hd.CROSS_WINDOW, 0
+    assert L.hd_decode_attn_final(*base, *bad, FAKE, ws, None) == hd.HD_ERR_INVALID_ARG
+    assert L.hd_decode_attn_final(*base[:4], 0, base[5], *ok, FAKE, ws, None) == hd.HD_ERR_INVALID_ARG
+
+
 def test_expand_rejects(lib):
     L = hd.lib()
     assert L.hd_expand_embed(FAKE, FAKE, FAKE, 1, 4, 2, 0, 8, 4, None) == hd.HD_ERR_INVALID_ARG

@@ -5,6 +5,7 @@ rewritten module, swaps its functions into the ``oracle`` package, and runs the
 pins that should fail. A mutant that every pin accepts would mean the pins do
 not constrain that part of the oracle.
 """
+import importlib
 import inspect
 import types
 
@@ -14,13 +15,21 @@ import oracle
 import oracle.attention
 import oracle.decode
 import oracle.expand
+import oracle.lm_head
+from tests import test_oracle_lm_head as lm_pins
 from tests import test_oracle_pins as pins
+from tests import test_oracle_rope as rope_pins
+
+# the package re-exports a function named `rope`, which hides the submodule attribute
+rope_mod = importlib.import_module("oracle.rope")
 
 EXPORTS = {
     oracle.attention: ["attn_bwd", "attn_bwd_dq_rows", "attn_bwd_kv_cols", "attn_fwd",
                        "attn_fwd_rows", "mask_matrix", "query_positions", "visible"],
     oracle.decode: ["decode_attn"],
     oracle.expand: ["expand_embed"],
+    oracle.lm_head: ["final_readout", "lm_head_ce", "lm_head_ce_rows"],
+    rope_mod: ["rope", "rope_expanded"],
 }
 
 
@@ -77,6 +86,26 @@ MUTANTS = [
     ("decode query at stream 0", oracle.decode, "qpos = T * n + streams",
      "qpos = T * n + 0 * streams",
      [(pins.test_golden_decode, "G")]),
+    ("readout of stream 0", oracle.lm_head, "return x[:, n - 1::n, :]", "return x[:, 0::n, :]",
+     [(lm_pins.test_readout_is_the_last_stream_of_each_token, 4)]),
+    ("loss sign flipped", oracle.lm_head, "loss = np.where(labels >= 0, lse - picked, 0.0)",
+     "loss = np.where(labels >= 0, picked - lse, 0.0)", [(lm_pins.test_ce_matches_torch_cross_entropy, None)]),
+    ("logsumexp without max", oracle.lm_head,
+     "lse = (mx + np.log(np.exp(logits - mx).sum(axis=-1, keepdims=True)))[..., 0]",
+     "lse = np.log(np.exp(logits).sum(axis=-1, keepdims=True))[..., 0]",
+     [(lm_pins.test_large_logits_stay_finite, None)]),
+    ("ignored label not zeroed", oracle.lm_head, "loss = np.where(labels >= 0, lse - picked, 0.0)",
+     "loss = lse - picked", [(lm_pins.test_ce_matches_torch_cross_entropy, None)]),
+    ("rope interleaved pairs", rope_mod,
+     "return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)",
+     "return np.stack([x[..., 0::2] * c - x[..., 1::2] * s, x[..., 1::2] * c + x[..., 0::2] * s], "
+     "axis=-1).reshape(x.shape)", [(rope_pins.test_first_pair_turns_by_exactly_p_radians, None)]),
+    ("rope sine sign", rope_mod, "x1 * c - x2 * s, x2 * c + x1 * s", "x1 * c + x2 * s, x2 * c - x1 * s",
+     [(rope_pins.test_first_pair_turns_by_exactly_p_radians, None)]),
+    ("rope frequency exponent i/D", rope_mod, "* 2.0 / D)", "* 1.0 / D)",
+     [(rope_pins.test_last_frequency_matches_its_closed_form, None)]),
+    ("rope at token index", rope_mod, "rope(k[b:b + 1], np.arange(S) + shift, base)",
+     "rope(k[b:b + 1], np.arange(S) // n + shift, base)", [(rope_pins.test_expanded_positions_are_physical, 4)]),
 ]
 
 
@@ -90,11 +119,11 @@ def test_pins_catch_mutant(case, golden, monkeypatch):
     if module is oracle.attention:
         # decode reads the mask predicate from the attention module
         monkeypatch.setattr(oracle.decode, "visible", mut.visible)
-    resolved = [(fn, (golden,) if a == "G" else (a,)) for fn, a in checks]
+    resolved = [(fn, (golden,) if a == "G" else () if a is None else (a,)) for fn, a in checks]
     assert _run_pins(golden, resolved), "planted mistake went unnoticed"
 
 
 def test_unmutated_oracle_passes_the_same_pins(golden):
     for case in MUTANTS:
         for fn, a in case[4]:
-            fn(*((golden,) if a == "G" else (a,)))
+            fn(*((golden,) if a == "G" else () if a is None else (a,)))

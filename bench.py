@@ -95,14 +95,16 @@ def step_plan(wl):
                         flops=4 * D * pr, pairs=pr, bytes=kv_bytes + io))
     ex_bytes = B * L * 4 + 2 * B * L * n * wl["d"] * 4
     ops.insert(0, dict(name="expand", kind="expand", flops=0, pairs=0, bytes=ex_bytes))
+    # final-stream LM-head cross-entropy: one GEMM of the B*L final rows with the head
+    ops.append(dict(name="lm_head_ce", kind="lm_head", flops=2 * B * L * wl["d"] * wl["V"], pairs=0))
     # rotary embedding of q and k in place: every element read and written once
     ops.append(dict(name="rope", kind="rope", flops=0, pairs=0, bytes=2 * 2 * B * S * (Hq + Hkv) * D))
     return ops
 
 
-LAUNCHES = {"expand": 1, "fwd": 1, "bwd": 3, "decode": 2, "decode_final": 2, "rope": 1}
+LAUNCHES = {"expand": 1, "fwd": 1, "bwd": 3, "decode": 2, "decode_final": 2, "rope": 1, "lm_head": 2}
 # operations measured on their own only (not part of the default hot-path step)
-EXTRA_KINDS = {"rope", "decode_final"}
+EXTRA_KINDS = {"rope", "decode_final", "lm_head"}
 
 # Extra workloads for per-configuration measurements (`--workload`); the
 # default is the whole hot-path step above.
@@ -122,6 +124,8 @@ WORKLOADS = {
                    ops=["expand"]),
     "decode8_final": dict(B=8, L=1, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=16384,
                           ops=["decode_final_cross_full", "decode_final_intra"]),
+    "lm_head": dict(B=2, L=8192, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=1,
+                    ops=["lm_head_ce"]),
     "rope": dict(B=1, L=32768, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=1,
                  ops=["rope"]),
 }
@@ -175,6 +179,10 @@ class Step:
             self.h["dq_new"] = syn.normal_bf16((B, n, Hq, D), 14)
         if "decode_final" in kinds:
             self.h["dq_fin"] = syn.normal_bf16((B, 1, Hq, D), 18)
+        if "lm_head" in kinds:
+            li = syn.lm_head_inputs(B, L, n, d, V, seed=19)
+            self.h["x_hid"] = li["x"]
+            self.h["labels"] = li["labels"]
         if "rope" in kinds and not attn:
             self.h["q"] = syn.normal_bf16((B, S, Hq, D), 16)
             self.h["k"] = syn.normal_bf16((B, S, Hkv, D), 17)
@@ -197,6 +205,12 @@ class Step:
             self.dec_o = {m: torch.empty_like(self.d["dq_new"]) for m in ("cross_full", "intra")}
             self.dec_l = {m: torch.empty((B, Hq, n), dtype=torch.float32, device=dev)
                           for m in ("cross_full", "intra")}
+        if "lm_head" in kinds:
+            self.w_head = torch.empty((V, d), dtype=torch.bfloat16, device=dev).normal_(0, 3.0 / math.sqrt(d), generator=g)
+            self.loss = torch.empty((B, L), dtype=torch.float32, device=dev)
+            self.loss_lse = torch.empty((B, L), dtype=torch.float32, device=dev)
+            self.ws_lm_n = hd.hd_lm_head_ce_workspace_bytes(B, L, V)
+            self.ws_lm = torch.empty(self.ws_lm_n, dtype=torch.uint8, device=dev)
         if "decode_final" in kinds:
             self.ws_fin_n = hd.hd_decode_final_workspace_bytes(B, n, T + 1, Hq, Hkv, D)
             self.ws_fin = torch.empty(self.ws_fin_n, dtype=torch.uint8, device=dev)
@@ -233,6 +247,8 @@ class Step:
             self.result.append(self.x[:, :1])
         elif "rope" in kinds:
             self.result.append(self.d["k"][:, :1])
+        elif "lm_head" in kinds:
+            self.result.append(self.loss)
         self.host_res = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in self.result]
         self.d2h_bytes = sum(t.numel() * t.element_size() for t in self.result)
 
@@ -244,6 +260,9 @@ class Step:
         name = op["name"]
         if op["kind"] == "expand":
             hd.hd_expand_embed(d["ids"], self.tables, self.x, B, L, n, wl["V"], wl["d"], 4, s)
+        elif op["kind"] == "lm_head":
+            hd.hd_lm_head_ce(d["x_hid"], self.w_head, d["labels"], self.loss, self.loss_lse, B, L, n,
+                             wl["d"], wl["V"], self.ws_lm, self.ws_lm_n, s)
         elif op["kind"] == "rope":
             hd.hd_rope_expanded(d["q"], d["k"], None, B, L, n, Hq, Hkv, D, 0, 10000.0, s)
         elif op["kind"] in ("fwd", "bwd"):
@@ -412,6 +431,8 @@ DESCRIPTIONS = {
     "expand": "expansion B4 L8192 n4, V32000, d4096 fp32 tables",
     "decode8_final": "final-stream-only decode (one query per sequence) CROSS_FULL + INTRA, B8 n4, "
                      "16384 prior tokens (65540 cache rows), Hq32 Hkv8 D128",
+    "lm_head": "final-stream readout + fused LM-head cross-entropy, x [2,32768,4096] bf16 (16384 final-stream "
+               "rows), head [32000,4096] bf16",
     "rope": "RoPE in place at physical positions, q [1,131072,32,128] + k [1,131072,8,128] bf16, base 10000",
 }
 
@@ -565,7 +586,7 @@ def main():
         rec = {"ms": round(m, 4)}
         if op["flops"]:
             rec["tflops"] = round(op["flops"] / (m * 1e-3) / 1e12, 1)
-            if op["kind"] in ("fwd", "bwd"):
+            if op["kind"] in ("fwd", "bwd", "lm_head"):
                 rec["frac_of_measured_bf16"] = round(rec["tflops"] / tf_peak, 4)
         if op.get("bytes"):
             rec["gbs"] = round(op["bytes"] / (m * 1e-3) / 1e9, 1)
@@ -573,7 +594,7 @@ def main():
         per_op[op["name"]] = rec
     dom = max(ops, key=lambda o: per_op[o["name"]]["ms"])
     dom_ms = per_op[dom["name"]]["ms"]
-    if dom["kind"] in ("fwd", "bwd"):
+    if dom["kind"] in ("fwd", "bwd", "lm_head"):
         ach = dom["flops"] / (dom_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": tf_peak, "unit": "TFLOP/s",
                 "frac": round(ach / tf_peak, 4),
@@ -588,7 +609,8 @@ def main():
              "decode": "hd_decode_attn (decode_split + decode_combine)",
              "expand": "hd_expand_embed (expand_kernel)",
              "decode_final": "hd_decode_attn_final (decode_split + decode_combine)",
-             "rope": "hd_rope_expanded (rope_kernel)"}[dom["kind"]]
+             "rope": "hd_rope_expanded (rope_kernel)",
+             "lm_head": "hd_lm_head_ce (lm_head_ce_kernel + lm_head_combine)"}[dom["kind"]]
     roof = {"kernel": f"{kname}, op {dom['name']}", **roof,
             "traffic": NCU_TRAFFIC.get((args.workload, dom["name"]))}
     if hbm_only:

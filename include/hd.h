@@ -114,6 +114,48 @@ int hd_rope_expanded(void* q, void* k, const int32_t* token_offset, int B, int L
                      int Hkv, int D, int final_stream_queries_only, double base, void* stream);
 
 /*
+ * hd_final_readout - the final stream's rows of the expanded sequence.
+ * Source: tahou.com page, "隐式序列缩放的技术细节" step 3 (the loss is taken
+ * only on the last stream of every token).
+ *
+ *   out[b, t, :] = x[b, t*n + n-1, :]        (exact copy of the bytes)
+ *
+ *   x    [B, n*L, d] elements of `elem_bytes` bytes; out [B, L, d]
+ * Supported: d * elem_bytes a multiple of 16.
+ */
+int hd_final_readout(const void* x, void* out, int B, int L, int n, int d, int elem_bytes,
+                     void* stream);
+
+/* Bytes of workspace hd_lm_head_ce needs (0 on invalid sizes). */
+size_t hd_lm_head_ce_workspace_bytes(int B, int L, int V);
+
+/*
+ * hd_lm_head_ce - LM-head cross-entropy on the final stream, fused.
+ * Source: tahou.com page, "隐式序列缩放的技术细节" step 3: only each token's
+ * last stream is supervised with the next-token loss; streams 0..n-2 get no
+ * direct supervision. The page gives no formula; this is the plain linear
+ * head and softmax cross-entropy:
+ *
+ *   h_r    = x[b, t*n + n-1, :]           (r = b*L + t; read in place)
+ *   lse_r  = ln sum_v exp(h_r . w_v)
+ *   loss_r = lse_r - h_r . w_{labels[r]}
+ *
+ *   x       bf16 [B, n*L, d]: hidden states of the expanded sequence
+ *   w       bf16 [V, d]: the LM head (no bias)
+ *   labels  int32 [B, L]: target of each token, already shifted by the caller;
+ *           a negative label marks a token without a target (loss 0). A
+ *           label >= V gives loss 0 and records HD_ERR_DEVICE_INDEX.
+ *   loss    fp32 [B, L]; lse fp32 [B, L] or NULL
+ * The logits are never written to memory: products are accumulated in fp32
+ * on the tensor cores and reduced to (max, sum of exp) per 256-wide
+ * vocabulary tile. Supported: d a multiple of 64.
+ * `workspace` must hold hd_lm_head_ce_workspace_bytes(B, L, V) bytes.
+ */
+int hd_lm_head_ce(const void* x, const void* w, const int32_t* labels, float* loss, float* lse,
+                  int B, int L, int n, int d, int V, void* workspace, size_t workspace_bytes,
+                  void* stream);
+
+/*
  * hd_attn_fwd - Stream-Factorized attention forward.
  * Source: tahou.com page, "规模化落地的工程优化" (intra / cross-stream bullets,
  * KV-mirror paragraph); "隐式序列缩放的技术细节" step 2 (causal attention).

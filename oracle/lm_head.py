@@ -49,7 +49,8 @@ def lm_head_ce_rows(x, w, labels, n, rows):
     """lm_head_ce for the flattened token indices `rows` (b*L + t) only."""
     B, S, d = x.shape
     L = S // n
-    h = _f64(final_readout(x, n)).reshape(B * L, d)[rows]
+    rows = np.asarray(rows, dtype=np.int64)
+    h = _f64(x[rows // L, (rows % L) * n + n - 1, :])  # token t of sequence b: position t*n + n-1
     w = _f64(w)
     lab = np.asarray(labels.cpu() if hasattr(labels, "cpu") else labels, dtype=np.int64).reshape(-1)[rows]
     logits = h @ w.T

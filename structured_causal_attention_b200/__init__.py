@@ -8,6 +8,9 @@ data-parallel hot path of Hidden Decoding with Stream-Factorized Attention
   at position (i-1)n+k);
 * ``hd_rope_expanded``  rotary position embedding of q and k at the physical
   positions p = t*n + s (continuous positions over the expanded sequence);
+* ``hd_final_readout`` / ``hd_lm_head_ce``  the final stream's hidden rows and the
+  LM-head cross-entropy on them (the only supervised stream), logits never
+  materialised;
 * ``hd_attn_fwd`` / ``hd_attn_bwd``  attention over the expanded sequence with
   intra-stream, cross-stream full-causal and cross-stream sliding-window masks,
   optionally with final-stream-only queries (KV-mirror);
@@ -40,6 +43,9 @@ from ._lib import (  # noqa: F401
     hd_decode_workspace_bytes,
     hd_device_status,
     hd_expand_embed,
+    hd_final_readout,
+    hd_lm_head_ce,
+    hd_lm_head_ce_workspace_bytes,
     hd_rope_expanded,
     lib,
     status_string,
@@ -168,3 +174,33 @@ def decode_attn_final(q, k_cache, v_cache, seqlen, n, mode, W=0, scale=None, str
     hd_decode_attn_final(q, k_cache, v_cache, seqlen, out, lse, B, n, Tcap, Hq, Hkv, D, mode, W,
                          scale, workspace, workspace.numel() * workspace.element_size(), stream)
     return out, lse
+
+
+def final_readout(x, n, stream=None):
+    """x [B, n*L, d] -> the final stream's rows [B, L, d] (positions t*n + n-1)."""
+    import torch
+
+    _need_cuda(x)
+    B, S, d = x.shape
+    L = S // n
+    out = torch.empty((B, L, d), dtype=x.dtype, device=x.device)
+    hd_final_readout(x, out, B, L, n, d, x.element_size(), stream)
+    return out
+
+
+def lm_head_ce(x, w, labels, n, stream=None, workspace=None):
+    """x bf16 [B, n*L, d], w bf16 [V, d], labels int32 [B, L] -> (loss, lse) fp32 [B, L]."""
+    import torch
+
+    _need_cuda(x, w, labels)
+    B, S, d = x.shape
+    L = S // n
+    V = w.shape[0]
+    loss = torch.empty((B, L), dtype=torch.float32, device=x.device)
+    lse = torch.empty((B, L), dtype=torch.float32, device=x.device)
+    nbytes = hd_lm_head_ce_workspace_bytes(B, L, V)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
+    hd_lm_head_ce(x, w, labels, loss, lse, B, L, n, d, V, workspace,
+                  workspace.numel() * workspace.element_size(), stream)
+    return loss, lse

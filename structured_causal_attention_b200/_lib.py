@@ -31,6 +31,9 @@ SIGNATURES = {
     "hd_version": (_I, []),
     "hd_expand_embed": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
     "hd_rope_expanded": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _D, _P]),
+    "hd_final_readout": (_I, [_P, _P, _I, _I, _I, _I, _I, _P]),
+    "hd_lm_head_ce_workspace_bytes": (_Z, [_I, _I, _I]),
+    "hd_lm_head_ce": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]),
     "hd_attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "hd_attn_bwd_workspace_bytes": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
     "hd_attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I,
@@ -109,6 +112,21 @@ def hd_rope_expanded(q, k, token_offset, B, L, n, Hq, Hkv, D, final_only, base, 
     return _check(lib().hd_rope_expanded(ptr(q), ptr(k), ptr(token_offset), B, L, n, Hq, Hkv, D,
                                          int(final_only), float(base), stream_handle(stream)),
                   "hd_rope_expanded")
+
+
+def hd_final_readout(x, out, B, L, n, d, elem_bytes, stream=None):
+    return _check(lib().hd_final_readout(ptr(x), ptr(out), B, L, n, d, elem_bytes,
+                                         stream_handle(stream)), "hd_final_readout")
+
+
+def hd_lm_head_ce_workspace_bytes(B, L, V):
+    return int(lib().hd_lm_head_ce_workspace_bytes(B, L, V))
+
+
+def hd_lm_head_ce(x, w, labels, loss, lse, B, L, n, d, V, workspace, workspace_bytes, stream=None):
+    return _check(lib().hd_lm_head_ce(ptr(x), ptr(w), ptr(labels), ptr(loss), ptr(lse), B, L, n, d,
+                                      V, ptr(workspace), workspace_bytes, stream_handle(stream)),
+                  "hd_lm_head_ce")
 
 
 def hd_attn_fwd(q, k, v, out, lse, B, L, n, Hq, Hkv, D, mode, W_tokens, final_only, scale,

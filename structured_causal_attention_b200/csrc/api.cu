@@ -260,6 +260,52 @@ int hd_rope_expanded(void* q, void* k, const int32_t* token_offset, int B, int L
   return from_cuda(launch_rope(p, static_cast<cudaStream_t>(stream)));
 }
 
+int hd_final_readout(const void* x, void* out, int B, int L, int n, int d, int elem_bytes,
+                     void* stream) {
+  if (!x || !out) return HD_ERR_INVALID_ARG;
+  if (B < 1 || L < 1 || n < 1 || d < 1) return HD_ERR_INVALID_ARG;
+  if (elem_bytes != 1 && elem_bytes != 2 && elem_bytes != 4 && elem_bytes != 8)
+    return HD_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out)) return HD_ERR_INVALID_ARG;
+  const long long row_bytes = static_cast<long long>(d) * elem_bytes;
+  if (row_bytes % 16 != 0) return HD_ERR_UNSUPPORTED;
+  return from_cuda(launch_final_readout(x, out, static_cast<long long>(B) * L, n, row_bytes,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+size_t hd_lm_head_ce_workspace_bytes(int B, int L, int V) {
+  if (B < 1 || L < 1 || V < 1) return 0;
+  return lm_head_workspace_bytes(static_cast<long long>(B) * L, V);
+}
+
+int hd_lm_head_ce(const void* x, const void* w, const int32_t* labels, float* loss, float* lse,
+                  int B, int L, int n, int d, int V, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  if (!x || !w || !labels || !loss || !workspace) return HD_ERR_INVALID_ARG;
+  if (B < 1 || L < 1 || n < 1 || d < 1 || V < 1) return HD_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(workspace)) return HD_ERR_INVALID_ARG;
+  if (d % 64 != 0) return HD_ERR_UNSUPPORTED;
+  const long long R = static_cast<long long>(B) * L;
+  if (R > (1LL << 31) - 1) return HD_ERR_UNSUPPORTED;
+  if (workspace_bytes < lm_head_workspace_bytes(R, V)) return HD_ERR_INVALID_ARG;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+    return HD_ERR_CUDA;
+  LmHeadParams p{};
+  p.labels = labels;
+  p.loss = loss;
+  p.lse = lse;
+  p.R = R;
+  p.V = V;
+  p.d = d;
+  const long long nvt = (V + 255) / 256;
+  p.part = static_cast<float*>(workspace);
+  p.pick = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(static_cast<size_t>(2 * nvt * R) * 4));
+  p.status = status_ptr();
+  return from_cuda(launch_lm_head_ce(p, x, w, n, sms, static_cast<cudaStream_t>(stream)));
+}
+
 int hd_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int L,
                 int n, int Hq, int Hkv, int D, int mode, int W_tokens,
                 int final_stream_queries_only, float scale, void* stream) {

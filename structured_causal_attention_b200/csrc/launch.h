@@ -51,6 +51,24 @@ struct RopeParams {
 };
 cudaError_t launch_rope(const RopeParams& p, cudaStream_t stream);
 
+struct LmHeadParams {
+  const int32_t* labels;  // [R]
+  float* loss;            // [R]
+  float* lse;             // [R] or null
+  float* part;            // [2][nvt][R]: per vocabulary tile max (log2 units), sum of exp2
+  float* pick;            // [R] logit of the label
+  int* status;
+  long long R;            // rows (tokens) = B*L
+  int V, d;
+  int nrb, nvt;           // row pairs, vocabulary tiles (set by the launcher)
+  long long units;
+};
+size_t lm_head_workspace_bytes(long long R, int V);
+cudaError_t launch_lm_head_ce(LmHeadParams p, const void* x, const void* w, int n, int num_sms,
+                              cudaStream_t stream);
+cudaError_t launch_final_readout(const void* x, void* out, long long rows, int n,
+                                 long long row_bytes, cudaStream_t stream);
+
 cudaError_t launch_expand(const int32_t* ids, const void* tables, void* out, int B, int L, int n,
                           int V, long long row_bytes, int* status, cudaStream_t stream);
 

@@ -95,6 +95,18 @@ def expand_inputs(B, L, n, V, d, seed=0, dtype=torch.float32, std=0.02):
     return {"ids": ids, "tables": tables}
 
 
+def lm_head_inputs(B, L, n, d, V, seed=0, ignore_every=0):
+    """Hidden states x bf16 [B, n*L, d] ~N(0, 1), LM head w bf16 [V, d] ~N(0, (3/sqrt(d))^2)
+    (logits of standard deviation about 3), labels int32 [B, L] uniform in [0, V); with
+    ``ignore_every`` = k > 0 every k-th label is -100 (a token without a target)."""
+    x = normal_bf16((B, n * L, d), seed * 16 + 11)
+    w = normal_bf16((V, d), seed * 16 + 12, std=3.0 / math.sqrt(d))
+    labels = token_ids(B, L, V, seed * 16 + 13)
+    if ignore_every:
+        labels.view(-1)[::ignore_every] = -100
+    return {"x": x, "w": w, "labels": labels}
+
+
 # Sizes of the workloads this library is exercised on.
 WORKLOADS = {
     # tiny end-to-end case: expansion + INTRA / CROSS_FULL fwd and bwd
@@ -105,6 +117,8 @@ WORKLOADS = {
     "cross_window": dict(B=2, L=8192, n=4, Hq=32, Hkv=8, D=128, W=1024, scale=1.0 / math.sqrt(128)),
     # long-context full cross-stream layer (+ final-stream-only queries)
     "long_cross": dict(B=1, L=32768, n=4, Hq=32, Hkv=8, D=128, scale=1.0 / math.sqrt(128)),
+    # final-stream LM-head loss over the cross_window layer's tokens (d = 32 heads x 128)
+    "lm_head": dict(B=2, L=8192, n=4, d=4096, V=32000),
     # multi-stream decode step against a 16384-token cache
     "decode": dict(B=8, n=4, T=16384, Hq=32, Hkv=8, D=128, scale=1.0 / math.sqrt(128)),
 }

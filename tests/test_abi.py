@@ -117,6 +117,27 @@ def test_decode_final_workspace_and_rejects(lib):
     assert L.hd_decode_attn_final(*base[:4], 0, base[5], *ok, FAKE, ws, None) == hd.HD_ERR_INVALID_ARG
 
 
+def test_lm_head_workspace_and_rejects(lib):
+    L = hd.lib()
+    ws = hd.hd_lm_head_ce_workspace_bytes(2, 100, 1000)
+    # per 256-wide vocabulary tile a (max, sum) pair per row, plus the label logit per row
+    assert ws == 4 * 2 * 200 * 4 + 1024
+    assert hd.hd_lm_head_ce_workspace_bytes(0, 100, 1000) == 0
+    ok = [FAKE, FAKE, FAKE, FAKE, 0, 2, 100, 4, 128, 1000, FAKE, ws, None]
+    def call(**kw):
+        a = list(ok)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return L.hd_lm_head_ce(*a)
+    assert call(a11=ws - 1) == hd.HD_ERR_INVALID_ARG
+    assert call(a0=0) == hd.HD_ERR_INVALID_ARG
+    assert call(a8=96) == hd.HD_ERR_UNSUPPORTED            # d not a multiple of 64
+    assert call(a1=FAKE + 4) == hd.HD_ERR_INVALID_ARG       # misaligned head
+    assert call(a9=0) == hd.HD_ERR_INVALID_ARG
+    assert L.hd_final_readout(FAKE, FAKE, 1, 4, 2, 6, 2, None) == hd.HD_ERR_UNSUPPORTED
+    assert L.hd_final_readout(0, FAKE, 1, 4, 2, 8, 2, None) == hd.HD_ERR_INVALID_ARG
+
+
 def test_expand_rejects(lib):
     L = hd.lib()
     assert L.hd_expand_embed(FAKE, FAKE, FAKE, 1, 4, 2, 0, 8, 4, None) == hd.HD_ERR_INVALID_ARG

@@ -16,7 +16,7 @@ Sources (page "微信WeLM提出Hidden Decoding：大模型推理新范式", taho
     mirror layers, so there only the final stream's queries exist and they read
     K/V built for all n streams.
 
-Readings where the page is not explicit (each one listed in the design doc):
+Readings where the page is not explicit:
   * a position is one of the "earlier positions" it may see (self included):
     the backbone is standard causal attention, and without self the first row of
     every stream would see nothing;

@@ -26,7 +26,10 @@
 //                   PV_0(j), S_0(j+1), PV_1(j), S_1(j+1)
 //               so one tile's MMAs run while the other tile's softmax works.
 //               S = Q K^T (M=128, N=128, both operands from shared memory);
-//               O += P V (M=128, N=D, P from TMEM, V MN-major from its TMA tile).
+//               O += P V (M=128, N=D, P from TMEM, V MN-major from its TMA tile),
+//               issued in two halves of 64 keys: the softmax signals P of keys
+//               64-127 before it reloads and exponentiates keys 0-63, so half
+//               of PV runs under the rest of the softmax.
 // MMAs from one thread execute in order, so when S_q(j) is complete, PV_q(j-1)
 // (issued before it) has finished reading P and updating O: the softmax may
 // then rescale O and overwrite P without another wait.
@@ -58,8 +61,8 @@ struct TcSmem {
   static constexpr int K_OFF = Q_OFF + 2 * Q_BYTES;        // 2 stages
   static constexpr int V_OFF = K_OFF + 2 * KV_BYTES;       // 2 stages
   static constexpr int BAR_OFF = V_OFF + 2 * KV_BYTES;
-  // q_full, k_full[2], v_full[2], kv_empty[2], s_full[2], p_full[2], o_final[2]
-  static constexpr int NBAR = 13;
+  // q_full, k_full[2], v_full[2], kv_empty[2], s_full[2], p_hi[2], p_lo[2], o_final[2]
+  static constexpr int NBAR = 15;
   static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;
   static constexpr int ABORT_OFF = SLOT_OFF + 4;
   static constexpr int USED = ABORT_OFF + 4 + 1024;
@@ -67,7 +70,8 @@ struct TcSmem {
   static constexpr int TOTAL = USED > 120 * 1024 ? USED : 120 * 1024;
 };
 
-enum { B_QF = 0, B_KF = 1, B_VF = 3, B_KE = 5, B_SF = 7, B_PF = 9, B_OF = 11 };
+// p_hi: P of keys 64-127 written; p_lo: P of keys 0-63 written
+enum { B_QF = 0, B_KF = 1, B_VF = 3, B_KE = 5, B_SF = 7, B_PA = 9, B_PB = 11, B_OF = 13 };
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -124,7 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     // softmax warps arrive once per warp (4); everything else arrives once
-    for (int i = 0; i < SM::NBAR; ++i) tc::mbar_init(bar(i), (i == B_PF || i == B_PF + 1) ? 4 : 1);
+    for (int i = 0; i < SM::NBAR; ++i) tc::mbar_init(bar(i), (i >= B_PA && i < B_PB + 2) ? 4 : 1);
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -193,17 +197,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int q = 0; q < 2 && ok; ++q) {
           if (in_range(q, j)) {
-            ok = tc::mbar_wait(bar(B_PF + q), pf_count[q] & 1, abort_flag, p.status);
+            // PV in two halves of 64 keys: keys 64-127 as soon as their P is
+            // written, while the softmax still works on keys 0-63
+            ok = tc::mbar_wait(bar(B_PA + q), pf_count[q] & 1, abort_flag, p.status);
             if (ok && !v_ready) ok = tc::mbar_wait(bar(B_VF + st), (i >> 1) & 1, abort_flag, p.status);
             if (!ok) break;
             v_ready = true;
+            tc::tc_fence_after();
+#pragma unroll
+            for (int kk = kBN / 32; kk < kBN / 16; ++kk)
+              tc::mma_ts(tmem + 256 * q + 128, tmem + 256 * q + 64 + kk * 8,
+                         tc::smem_desc_sw128(sV + st * SM::KV_BYTES + kk * 2048, kSub, 1024), idO,
+                         (j > lo[q] || kk > kBN / 32) ? 1u : 0u);
+            ok = tc::mbar_wait(bar(B_PB + q), pf_count[q] & 1, abort_flag, p.status);
+            if (!ok) break;
             ++pf_count[q];
             tc::tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < kBN / 16; ++kk)
+            for (int kk = 0; kk < kBN / 32; ++kk)
               tc::mma_ts(tmem + 256 * q + 128, tmem + 256 * q + 64 + kk * 8,
-                         tc::smem_desc_sw128(sV + st * SM::KV_BYTES + kk * 2048, kSub, 1024), idO,
-                         (j > lo[q] || kk > 0) ? 1u : 0u);
+                         tc::smem_desc_sw128(sV + st * SM::KV_BYTES + kk * 2048, kSub, 1024), idO, 1u);
             if (j == hi[q]) tc::mma_commit(bar(B_OF + q));
           }
           if (in_range(q, j + 1)) {
@@ -305,6 +318,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
       exp_half(v1, 1, m_use);
+      tc::tmem_wait_st();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar(B_PA + q));
       {
         uint32_t v[64];
         tc::tmem_ld32(tS, v);
@@ -316,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tmem_wait_st();
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(bar(B_PF + q));
+      if (lane == 0) tc::mbar_arrive(bar(B_PB + q));
     }
     const bool has_rows = my_lo <= my_hi;
     if (ok && has_rows && !*abort_flag) ok = tc::mbar_wait(bar(B_OF + q), 0, abort_flag, p.status);

@@ -121,3 +121,40 @@ def test_fwd_final_only_matches_full_rows():
         o_fin, l_fin = run_fwd(fin, n, mode, W, 1, 0.09)
         check(host64(o_fin), host64(o_all[:, n - 1::n]), 1e-2, 1e-4, "final rows")
         check(host64(l_fin), host64(l_all[:, :, n - 1::n]), 1e-4, 1e-5, "final lse")
+
+
+@pytest.mark.parametrize("mode", MODES, ids=["INTRA", "CROSS_FULL", "CROSS_WINDOW"])
+@pytest.mark.parametrize("fin", [0, 1], ids=["all", "final"])
+def test_fwd_scores_rising_along_the_keys(mode, fin):
+    """Scores grow by ~14 (log2 units) per 32 keys, so the running max of every
+    row is raised inside tiles, not only on its first chunk: exercises the
+    on-the-spot rescale of O, l and the P chunks already written."""
+    need_gpu()
+    B, L, n, Hq, Hkv, D, W = 1, 96, 4, 2, 1, 64, 40
+    S = n * L
+    g = torch.Generator().manual_seed(7)
+    q = torch.zeros(B, L if fin else S, Hq, D)
+    q[..., 0] = 1.0
+    q[..., 1:] = 0.1 * torch.randn(q[..., 1:].shape, generator=g)
+    k = 0.1 * torch.randn(B, S, Hkv, D, generator=g)
+    k[..., 0] = 0.3 * torch.arange(S, dtype=torch.float32)[None, :, None]
+    v = torch.randn(B, S, Hkv, D, generator=g)
+    inp = {"q": q.bfloat16(), "k": k.bfloat16(), "v": v.bfloat16()}
+    out, lse = run_fwd(inp, n, mode, W, fin, 1.0)
+    o_ref, l_ref = oracle.attn_fwd(inp["q"], inp["k"], inp["v"], n, mode, W, bool(fin), 1.0)
+    check(host64(out), o_ref, O_MAX, O_MEAN, "O")
+    check(host64(lse), l_ref, LSE_MAX * 40, LSE_MAX * 40, "LSE")  # |LSE| reaches ~115 here
+
+
+def test_fwd_spiky_scores():
+    """Q and K ~N(0, 3^2): scaled scores of standard deviation ~9, near one-hot rows
+    (V stays ~N(0, 1), so the bf16 rounding of P keeps the usual output bound)."""
+    need_gpu()
+    B, L, n, Hq, Hkv, D = 1, 70, 4, 4, 2, 128
+    inp = syn.attention_inputs(B, L, n, Hq, Hkv, D, seed=9)
+    inp = {key: ((val.float() * 3.0).bfloat16() if key in ("q", "k") else val) for key, val in inp.items()}
+    for mode in MODES:
+        out, lse = run_fwd(inp, n, mode, 7, 0, 1.0 / math.sqrt(D))
+        o_ref, l_ref = oracle.attn_fwd(inp["q"], inp["k"], inp["v"], n, mode, 7, False, 1.0 / math.sqrt(D))
+        check(host64(out), o_ref, O_MAX, O_MEAN, "O")
+        check(host64(lse), l_ref, LSE_MAX * 4, LSE_MAX * 4, "LSE")

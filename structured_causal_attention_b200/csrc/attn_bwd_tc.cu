@@ -24,7 +24,11 @@
 //               bulk reduce-add (the TMA unit does the adds, not the SM).
 //   warp 12     TMA: K, V once; Q and dO tiles (3 stages) plus the tile's
 //               packed LSE and D rows (bulk copies).
-//   warp 13     TMEM allocation; lane 0 issues the MMAs.
+//   warp 13     TMEM allocation; lane 0 issues dV, dK and dQ^T.
+//   warp 14     lane 0 issues S^T and dP^T of the next tile.
+// One thread issues a tcgen05.mma only every ~75 cycles, more than twice what
+// an N=64 MMA takes to run, so the two groups get an issuer each; their
+// hand-offs go through the barriers below, not through issue order.
 // Every mbarrier wait is bounded (HD_ERR_TIMEOUT, then every role leaves).
 #include <cuda.h>
 
@@ -39,7 +43,7 @@ namespace {
 constexpr int kKN = 128;   // keys per CTA
 constexpr int kQM = 64;    // query rows per iteration
 constexpr int kQS = 3;     // Q / dO stages
-constexpr int kThreads = 448;
+constexpr int kThreads = 480;
 constexpr uint32_t kTmemCols = 512;
 
 template <int D>
@@ -70,7 +74,7 @@ struct BtSmem {
 enum {
   B_KV = 0,   // K and V loaded
   B_QF = 1,   // [kQS] Q, dO and the packed LSE / D rows of a stage loaded
-  B_QE = 4,   // [kQS] stage free (MMA commit)
+  B_QE = 4,   // [kQS] stage free (one MMA commit from each issuer)
   B_SF = 7,   // [2] S^T / dP^T ready (MMA commit)
   B_PF = 9,   // P^T / dS^T written (8 warp arrivals)
   B_PE = 10,  // P^T / dS^T consumed by the MMAs (MMA commit)
@@ -131,6 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < SM::NBAR; ++i) {
       uint32_t cnt = 1;
       if (i == B_DE || i == B_DE + 1) cnt = 4;
+      if (i >= B_QE && i < B_QE + kQS) cnt = 2;
       if (i == B_PF) cnt = 8;
       tc::mbar_init(bar(i), cnt);
     }
@@ -177,8 +182,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::bulk_load(sbase + SM::DL_OFF + st * kQM * 4, p.deltap + pk, kQM * 4, bar(B_QF + st));
       }
     }
-  } else if (warp == 13) {
-    // ------------------------------------------------------------- MMA issuer
+  } else if (warp == 13 || warp == 14) {
+    // ------------------------------------------------------------ MMA issuers
     if (lane == 0 && total > 0) {
       constexpr uint32_t idSP = tc::idesc_bf16_f32(128, kQM, 0, 0);  // S^T, dP^T
       constexpr uint32_t idKV = tc::idesc_bf16_f32(128, D, 0, 1);    // dV, dK
@@ -194,58 +199,58 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dSm = tc::smem_desc_sw128(sDS, SM::QSUB, 1024);
       const uint64_t dKt = tc::smem_desc_sw128(sK, kt_lbo, 1024);
       auto add = [](uint64_t d, uint32_t bytes) { return d + (bytes >> 4); };
-      auto issue_sp = [&](int buf, int st) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ko = (kk >> 2) * SM::KSUB + (kk & 3) * 32;
-          const uint32_t qo = (st * NSUB + (kk >> 2)) * SM::QSUB + (kk & 3) * 32;
-          tc::mma_ss(tmem + 128 * buf, add(dK, ko), add(dQk, qo), idSP, kk > 0);
-          tc::mma_ss(tmem + 128 * buf + 64, add(dV, ko), add(dOk, qo), idSP, kk > 0);
-        }
-      };
-      bool ok = tc::mbar_wait(bar(B_KV), 0, abort_flag, p.status) &&
-                tc::mbar_wait(bar(B_QF), 0, abort_flag, p.status);
-      if (ok) {
-        tc::tc_fence_after();
-        issue_sp(0, 0);
-        tc::mma_commit(bar(B_SF));
-      }
-      for (int it = 0; ok && it < total; ++it) {
-        const int x = it & 1, st = it % kQS;
-        if (it + 1 < total) {
-          const int x1 = (it + 1) & 1, s1 = (it + 1) % kQS;
-          ok = tc::mbar_wait(bar(B_QF + s1), ((it + 1) / kQS) & 1, abort_flag, p.status);
-          if (ok && it + 1 >= 2)
-            ok = tc::mbar_wait(bar(B_DE + x1), (((it + 1) >> 1) - 1) & 1, abort_flag, p.status);
+      bool ok = tc::mbar_wait(bar(B_KV), 0, abort_flag, p.status);
+      if (warp == 14) {
+        // S^T, dP^T of tile it into TMEM buffer it & 1, once the stage is
+        // loaded and dQ^T of tile it-2 (same buffer) has been read out
+        for (int it = 0; ok && it < total; ++it) {
+          const int x = it & 1, st = it % kQS;
+          ok = tc::mbar_wait(bar(B_QF + st), (it / kQS) & 1, abort_flag, p.status);
+          if (ok && it >= 2) ok = tc::mbar_wait(bar(B_DE + x), ((it >> 1) - 1) & 1, abort_flag, p.status);
           if (!ok) break;
           tc::tc_fence_after();
-          issue_sp(x1, s1);
-          tc::mma_commit(bar(B_SF + x1));
-        }
-        ok = tc::mbar_wait(bar(B_PF), it & 1, abort_flag, p.status);
-        if (!ok) break;
-        tc::tc_fence_after();
-        const uint32_t acc = it > 0 ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < kQM / 16; ++kk) {  // reduce over the 64 queries
-          const uint64_t ap = add(dP, kk * 32);
-          const uint64_t as = add(dS, kk * 32);
-          const uint64_t bo = add(dOm, st * NSUB * SM::QSUB + kk * 2048);
-          const uint64_t bq = add(dQm, st * NSUB * SM::QSUB + kk * 2048);
-          tc::mma_ss(tdV, ap, bo, idKV, (acc | kk) ? 1u : 0u);
-          tc::mma_ss(tdK, as, bq, idKV, (acc | kk) ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t ko = (kk >> 2) * SM::KSUB + (kk & 3) * 32;
+            const uint32_t qo = (st * NSUB + (kk >> 2)) * SM::QSUB + (kk & 3) * 32;
+            tc::mma_ss(tmem + 128 * x, add(dK, ko), add(dQk, qo), idSP, kk > 0);
+            tc::mma_ss(tmem + 128 * x + 64, add(dV, ko), add(dOk, qo), idSP, kk > 0);
+          }
+          tc::mma_commit(bar(B_SF + x));
+          tc::mma_commit(bar(B_QE + st));
         }
+      } else {
+        // dV, dK, dQ^T of tile it once P^T / dS^T are written
+        for (int it = 0; ok && it < total; ++it) {
+          const int x = it & 1, st = it % kQS;
+          ok = tc::mbar_wait(bar(B_QF + st), (it / kQS) & 1, abort_flag, p.status) &&
+               tc::mbar_wait(bar(B_PF), it & 1, abort_flag, p.status);
+          if (!ok) break;
+          tc::tc_fence_after();
+          const uint32_t acc = it > 0 ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < kKN / 16; ++kk) {  // reduce over the 128 keys
-          const uint64_t ak = add(dKt, kk * 2048);
-          const uint64_t bs = add(dSm, kk * 2048);
-          tc::mma_ss(tmem + 128 * x, ak, bs, idDQ, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < kQM / 16; ++kk) {  // reduce over the 64 queries
+            const uint64_t ap = add(dP, kk * 32);
+            const uint64_t as = add(dS, kk * 32);
+            const uint64_t bo = add(dOm, st * NSUB * SM::QSUB + kk * 2048);
+            const uint64_t bq = add(dQm, st * NSUB * SM::QSUB + kk * 2048);
+            tc::mma_ss(tdV, ap, bo, idKV, (acc | kk) ? 1u : 0u);
+            tc::mma_ss(tdK, as, bq, idKV, (acc | kk) ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < kKN / 16; ++kk) {  // reduce over the 128 keys
+            const uint64_t ak = add(dKt, kk * 2048);
+            const uint64_t bs = add(dSm, kk * 2048);
+            tc::mma_ss(tmem + 128 * x, ak, bs, idDQ, kk > 0 ? 1u : 0u);
+          }
+          tc::mma_commit(bar(B_DF + x));
+          tc::mma_commit(bar(B_QE + st));
+          tc::mma_commit(bar(B_PE));
         }
-        tc::mma_commit(bar(B_DF + x));
-        tc::mma_commit(bar(B_QE + st));
-        tc::mma_commit(bar(B_PE));
+        // every S^T / dP^T MMA finished before the last P^T was written, so this
+        // covers both issuers
+        tc::mma_commit(bar(B_END));
       }
-      tc::mma_commit(bar(B_END));
     }
   } else if (warp < 8) {
     // ------------------------- P^T, dS^T: one key per thread, warpgroup sw takes

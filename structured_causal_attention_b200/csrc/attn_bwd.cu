@@ -22,42 +22,56 @@ namespace hd {
 
 namespace {
 
-__global__ void bwd_pre_kernel(const AttnParams p) {
+// D = rowsum(dO * O) and LSE * log2(e), packed per problem; the fp32 dQ
+// accumulator zeroed. D/8 lanes per row (16-byte loads of 8 bf16 each), so a
+// warp covers 32 / (D/8) rows per pass.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const AttnParams p) {
+  constexpr int LPR = D / 8;           // lanes per row
+  constexpr int RPW = 32 / LPR;        // rows per warp
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long row = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + warp;
+  const int sub = lane / LPR, sl = lane % LPR;
+  const long long row = (static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + warp) * RPW + sub;
   const long long total = static_cast<long long>(p.B) * p.Sq * p.Hq;
-  if (row >= total) return;
+  const bool valid = row < total;
+  float acc = 0.f;
+  if (valid) {
+    const uint4 ov = __ldcs(reinterpret_cast<const uint4*>(p.o + row * D) + sl);
+    const uint4 gv = __ldcs(reinterpret_cast<const uint4*>(p.dout + row * D) + sl);
+    const uint32_t* o2 = reinterpret_cast<const uint32_t*>(&ov);
+    const uint32_t* g2 = reinterpret_cast<const uint32_t*>(&gv);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float2 of = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o2[w]));
+      const float2 gf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&g2[w]));
+      acc = fmaf(of.x, gf.x, acc);
+      acc = fmaf(of.y, gf.y, acc);
+    }
+  }
+#pragma unroll
+  for (int s = LPR / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+  if (!valid) return;
   const int h = static_cast<int>(row % p.Hq);
   const long long bi = row / p.Hq;
   const long long i = bi % p.Sq, b = bi / p.Sq;
-  const __nv_bfloat16* o = p.o + row * p.D;
-  const __nv_bfloat16* g = p.dout + row * p.D;
-  float acc = 0.f;
-  for (int c = lane * 2; c < p.D; c += 64) {
-    const __nv_bfloat162 ov = *reinterpret_cast<const __nv_bfloat162*>(o + c);
-    const __nv_bfloat162 gv = *reinterpret_cast<const __nv_bfloat162*>(g + c);
-    acc = fmaf(__low2float(ov), __low2float(gv), acc);
-    acc = fmaf(__high2float(ov), __high2float(gv), acc);
-  }
-#pragma unroll
-  for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
   // packed row statistics of problem (b, h, grp), row r
   const bool intra_groups = p.mode == HD_INTRA && !p.final_only;
   const long long grp = intra_groups ? i % p.n : 0;
   const long long r = intra_groups ? i / p.n : i;
   const long long pk = ((b * p.Hq + h) * p.groups + grp) * p.lq_pad;
-  if (lane == 0) {
+  if (sl == 0) {
     p.deltap[pk + r] = acc;
     p.lse2p[pk + r] = p.lse[(b * p.Hq + h) * p.Sq + i] * 1.4426950408889634074f;
   }
   if (r == p.Lq - 1) {  // zero the padding rows after the problem's last row
-    for (int j = lane; j < p.lq_pad - p.Lq; j += 32) {
+    for (int j = sl; j < p.lq_pad - p.Lq; j += LPR) {
       p.deltap[pk + p.Lq + j] = 0.f;
       p.lse2p[pk + p.Lq + j] = 0.f;
     }
   }
-  float4* z = reinterpret_cast<float4*>(p.dq_acc + row * p.D);
-  for (int c = lane; c < p.D / 4; c += 32) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+  float4* z = reinterpret_cast<float4*>(p.dq_acc + row * D) + 2 * sl;
+  z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+  z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // INTRA with final-stream-only queries: only stream n-1's keys are read, so
@@ -95,7 +109,10 @@ __global__ void bwd_dq_kernel(const AttnParams p, long long n8) {
 cudaError_t launch_attn_bwd(const AttnParams& p, cudaStream_t stream) {
   if (p.D != 64 && p.D != 128) return cudaErrorInvalidValue;
   const long long rows = static_cast<long long>(p.B) * p.Sq * p.Hq;
-  bwd_pre_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(p);
+  const long long rows_per_block = 8 * (32 / (p.D / 8));  // 8 warps
+  const unsigned pre_blocks = static_cast<unsigned>((rows + rows_per_block - 1) / rows_per_block);
+  if (p.D == 64) bwd_pre_kernel<64><<<pre_blocks, 256, 0, stream>>>(p);
+  else bwd_pre_kernel<128><<<pre_blocks, 256, 0, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = launch_attn_bwd_tc_main(p, stream);

@@ -276,6 +276,17 @@ int hd_decode_attn_noalloc(const void* q, const void* k_cache, const void* v_cac
                            void* stream);
 
 /*
+ * hd_selftest_wait_timeout - test the bounded-wait failure path (no fault).
+ * Launches one thread that waits, through the same bounded wait the
+ * tensor-core kernels use, on a barrier nothing will complete, giving up after
+ * `limit_cycles` SM cycles (1 .. 2^33). Afterwards the device status word reads
+ * HD_ERR_TIMEOUT (hd_device_status), and until it is cleared the tensor-core
+ * kernels (hd_attn_fwd, hd_attn_bwd, hd_lm_head_ce) return without doing their
+ * work, as they would after a real timeout.
+ */
+int hd_selftest_wait_timeout(long long limit_cycles, void* stream);
+
+/*
  * Read (and, if `clear` is non-zero, reset) the device status word of the
  * current device. Synchronizes `stream` first. Returns HD_OK when no kernel
  * recorded an error since the last clear, else the first recorded code.

@@ -47,6 +47,7 @@ from ._lib import (  # noqa: F401
     hd_lm_head_ce,
     hd_lm_head_ce_workspace_bytes,
     hd_rope_expanded,
+    hd_selftest_wait_timeout,
     lib,
     status_string,
 )

@@ -46,6 +46,7 @@ SIGNATURES = {
                                   _Z, _P]),
     "hd_decode_attn_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F,
                                     _P]),
+    "hd_selftest_wait_timeout": (_I, [ctypes.c_longlong, _P]),
     "hd_device_status": (_I, [_P, _I]),
 }
 
@@ -180,6 +181,11 @@ def hd_decode_attn_noalloc(q, k_cache, v_cache, seqlen, out, lse, B, n, Tcap, Hq
                                                ptr(out), ptr(lse), B, n, Tcap, Hq, Hkv, D, mode,
                                                W_tokens, float(scale), stream_handle(stream)),
                   "hd_decode_attn_noalloc")
+
+
+def hd_selftest_wait_timeout(limit_cycles, stream=None):
+    return _check(lib().hd_selftest_wait_timeout(int(limit_cycles), stream_handle(stream)),
+                  "hd_selftest_wait_timeout")
 
 
 def hd_device_status(stream=None, clear=True):

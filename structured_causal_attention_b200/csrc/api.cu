@@ -381,6 +381,11 @@ int hd_decode_attn_final(const void* q, const void* k_cache, const void* v_cache
                          W_tokens, 1, scale, workspace, workspace_bytes, stream);
 }
 
+int hd_selftest_wait_timeout(long long limit_cycles, void* stream) {
+  if (limit_cycles < 1 || limit_cycles > (1LL << 33)) return HD_ERR_INVALID_ARG;
+  return from_cuda(launch_wait_timeout(limit_cycles, status_ptr(), static_cast<cudaStream_t>(stream)));
+}
+
 int hd_device_status(void* stream, int clear) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return HD_ERR_CUDA;
   int* ptr = status_ptr();

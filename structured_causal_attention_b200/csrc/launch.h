@@ -69,6 +69,8 @@ cudaError_t launch_lm_head_ce(LmHeadParams p, const void* x, const void* w, int 
 cudaError_t launch_final_readout(const void* x, void* out, long long rows, int n,
                                  long long row_bytes, cudaStream_t stream);
 
+cudaError_t launch_wait_timeout(long long limit_cycles, int* status, cudaStream_t stream);
+
 cudaError_t launch_expand(const int32_t* ids, const void* tables, void* out, int B, int L, int n,
                           int V, long long row_bytes, int* status, cudaStream_t stream);
 

@@ -165,6 +165,12 @@ def test_rope_rejects(lib):
     assert call(a8=512) == hd.HD_ERR_UNSUPPORTED
 
 
+def test_selftest_rejects_bad_limits(lib):
+    L = hd.lib()
+    assert L.hd_selftest_wait_timeout(0, None) == hd.HD_ERR_INVALID_ARG
+    assert L.hd_selftest_wait_timeout((1 << 33) + 1, None) == hd.HD_ERR_INVALID_ARG
+
+
 def test_python_binding_raises_on_error(lib):
     with pytest.raises(hd.HDError) as e:
         hd.hd_attn_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 4, 4, 2, 96, 0, 1, 0, 0.1, stream=0)

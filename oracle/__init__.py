@@ -28,4 +28,4 @@ from .attention import (  # noqa: F401
 from .decode import decode_attn  # noqa: F401
 from .expand import expand_embed  # noqa: F401
 from .rope import rope, rope_expanded  # noqa: F401
-from .lm_head import final_readout, lm_head_ce, lm_head_ce_rows  # noqa: F401
+from .lm_head import final_readout, lm_head_ce, lm_head_ce_grad, lm_head_ce_rows  # noqa: F401

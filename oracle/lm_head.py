@@ -58,3 +58,28 @@ def lm_head_ce_rows(x, w, labels, n, rows):
     lse = (mx + np.log(np.exp(logits - mx).sum(axis=-1, keepdims=True)))[:, 0]
     picked = logits[np.arange(len(rows)), np.clip(lab, 0, w.shape[0] - 1)]
     return np.where(lab >= 0, lse - picked, 0.0), lse
+
+
+def lm_head_ce_grad(x, w, labels, n):
+    """Gradients of the summed loss, sum_r loss_r (ignored tokens add nothing).
+
+    With G = softmax(logits) - onehot(label) per supervised row (G = 0 for a
+    negative label), the chain rule gives dh = G W and dW = G^T h. Returns
+    (G [B, L, V], dh [B, L, d], dW [V, d]) in float64; dh is the gradient with
+    respect to the final-stream rows, i.e. dX[b, t*n + n-1] = dh[b, t] and the
+    other streams' rows of dX are zero.
+    """
+    h = _f64(final_readout(x, n))                     # [B, L, d]
+    w = _f64(w)
+    labels = np.asarray(labels.cpu() if hasattr(labels, "cpu") else labels, dtype=np.int64)
+    logits = h @ w.T
+    mx = logits.max(axis=-1, keepdims=True)
+    p = np.exp(logits - mx)
+    p /= p.sum(axis=-1, keepdims=True)
+    g = p.copy()
+    rows = np.argwhere(labels >= 0)
+    g[rows[:, 0], rows[:, 1], labels[labels >= 0]] -= 1.0
+    g[labels < 0] = 0.0
+    dh = g @ w
+    dw = np.einsum("blv,bld->vd", g, h)
+    return g, dh, dw

@@ -89,3 +89,50 @@ def test_rows_helper_matches_full():
     rl, rs = oracle.lm_head_ce_rows(x, w, labels, n, rows)
     np.testing.assert_allclose(rl, loss.reshape(-1)[rows], atol=1e-13)
     np.testing.assert_allclose(rs, lse.reshape(-1)[rows], atol=1e-13)
+
+
+def test_grad_matches_central_differences():
+    """dh and dW of the summed loss against float64 central differences."""
+    B, L, n, d, V = 1, 3, 2, 5, 7
+    x, w = _rand((B, n * L, d), 11), _rand((V, d), 12)
+    labels = np.array([[2, -1, 6]])
+    _, dh, dw = oracle.lm_head_ce_grad(x, w, labels, n)
+    eps = 1e-6
+
+    def total(xx, ww):
+        return oracle.lm_head_ce(xx, ww, labels, n)[0].sum()
+    for (t, k) in [(0, 0), (0, 4), (1, 2), (2, 3)]:
+        xp, xm = x.copy(), x.copy()
+        xp[0, t * n + n - 1, k] += eps
+        xm[0, t * n + n - 1, k] -= eps
+        num = (total(xp, w) - total(xm, w)) / (2 * eps)
+        assert abs(num - dh[0, t, k]) < 1e-7, (t, k, num, dh[0, t, k])
+    for (v, k) in [(0, 0), (2, 1), (6, 4), (3, 2)]:
+        wp, wm = w.copy(), w.copy()
+        wp[v, k] += eps
+        wm[v, k] -= eps
+        num = (total(x, wp) - total(x, wm)) / (2 * eps)
+        assert abs(num - dw[v, k]) < 1e-7, (v, k, num, dw[v, k])
+    # the unsupervised streams' rows get no gradient: a change there changes nothing
+    xs = x.copy()
+    xs[0, 0, :] += 1.0
+    assert total(xs, w) == total(x, w)
+
+
+def test_grad_rows_sum_to_zero_and_zero_head_closed_form():
+    B, L, n, d, V = 2, 4, 3, 6, 9
+    x = _rand((B, n * L, d), 13)
+    labels = np.array([[0, 8, -100, 4], [1, 1, 2, 3]])
+    g, _, _ = oracle.lm_head_ce_grad(x, _rand((V, d), 14), labels, n)
+    sup = labels >= 0
+    np.testing.assert_allclose(g[sup].sum(axis=-1), 0.0, atol=1e-14)
+    assert (g[~sup] == 0).all()
+    g0, dh0, dw0 = oracle.lm_head_ce_grad(x, np.zeros((V, d)), labels, n)
+    want = np.full((B, L, V), 1.0 / V)
+    want[~sup] = 0
+    for b in range(B):
+        for t in range(L):
+            if labels[b, t] >= 0:
+                want[b, t, labels[b, t]] -= 1.0
+    np.testing.assert_allclose(g0, want, atol=1e-15)
+    assert (dh0 == 0).all()

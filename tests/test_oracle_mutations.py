@@ -28,7 +28,7 @@ EXPORTS = {
                        "attn_fwd_rows", "mask_matrix", "query_positions", "visible"],
     oracle.decode: ["decode_attn"],
     oracle.expand: ["expand_embed"],
-    oracle.lm_head: ["final_readout", "lm_head_ce", "lm_head_ce_rows"],
+    oracle.lm_head: ["final_readout", "lm_head_ce", "lm_head_ce_grad", "lm_head_ce_rows"],
     rope_mod: ["rope", "rope_expanded"],
 }
 
@@ -96,6 +96,10 @@ MUTANTS = [
      [(lm_pins.test_large_logits_stay_finite, None)]),
     ("ignored label not zeroed", oracle.lm_head, "loss = np.where(labels >= 0, lse - picked, 0.0)",
      "loss = lse - picked", [(lm_pins.test_ce_matches_torch_cross_entropy, None)]),
+    ("CE gradient without the one-hot", oracle.lm_head, "g[rows[:, 0], rows[:, 1], labels[labels >= 0]] -= 1.0",
+     "pass", [(lm_pins.test_grad_matches_central_differences, None)]),
+    ("dW from the probabilities", oracle.lm_head, 'dw = np.einsum("blv,bld->vd", g, h)',
+     'dw = np.einsum("blv,bld->vd", p, h)', [(lm_pins.test_grad_matches_central_differences, None)]),
     ("rope interleaved pairs", rope_mod,
      "return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)",
      "return np.stack([x[..., 0::2] * c - x[..., 1::2] * s, x[..., 1::2] * c + x[..., 0::2] * s], "

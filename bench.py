@@ -97,14 +97,17 @@ def step_plan(wl):
     ops.insert(0, dict(name="expand", kind="expand", flops=0, pairs=0, bytes=ex_bytes))
     # final-stream LM-head cross-entropy: one GEMM of the B*L final rows with the head
     ops.append(dict(name="lm_head_ce", kind="lm_head", flops=2 * B * L * wl["d"] * wl["V"], pairs=0))
+    # its gradients: logits recomputed, dh = G W, dW = G^T h (three GEMMs of the same size)
+    ops.append(dict(name="lm_head_ce_bwd", kind="lm_head_bwd", flops=3 * 2 * B * L * wl["d"] * wl["V"], pairs=0))
     # rotary embedding of q and k in place: every element read and written once
     ops.append(dict(name="rope", kind="rope", flops=0, pairs=0, bytes=2 * 2 * B * S * (Hq + Hkv) * D))
     return ops
 
 
-LAUNCHES = {"expand": 1, "fwd": 1, "bwd": 3, "decode": 2, "decode_final": 2, "rope": 1, "lm_head": 2}
+LAUNCHES = {"expand": 1, "fwd": 1, "bwd": 3, "decode": 2, "decode_final": 2, "rope": 1, "lm_head": 2,
+            "lm_head_bwd": 3}
 # operations measured on their own only (not part of the default hot-path step)
-EXTRA_KINDS = {"rope", "decode_final", "lm_head"}
+EXTRA_KINDS = {"rope", "decode_final", "lm_head", "lm_head_bwd"}
 
 # Extra workloads for per-configuration measurements (`--workload`); the
 # default is the whole hot-path step above.
@@ -126,6 +129,8 @@ WORKLOADS = {
                           ops=["decode_final_cross_full", "decode_final_intra"]),
     "lm_head": dict(B=2, L=8192, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=1,
                     ops=["lm_head_ce"]),
+    "lm_head_train": dict(B=2, L=8192, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=1,
+                          ops=["lm_head_ce", "lm_head_ce_bwd"]),
     "rope": dict(B=1, L=32768, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=1,
                  ops=["rope"]),
 }
@@ -179,7 +184,7 @@ class Step:
             self.h["dq_new"] = syn.normal_bf16((B, n, Hq, D), 14)
         if "decode_final" in kinds:
             self.h["dq_fin"] = syn.normal_bf16((B, 1, Hq, D), 18)
-        if "lm_head" in kinds:
+        if kinds & {"lm_head", "lm_head_bwd"}:
             li = syn.lm_head_inputs(B, L, n, d, V, seed=19)
             self.h["x_hid"] = li["x"]
             self.h["labels"] = li["labels"]
@@ -208,12 +213,17 @@ class Step:
             self.dec_o = {m: torch.empty_like(self.d["dq_new"]) for m in ("cross_full", "intra")}
             self.dec_l = {m: torch.empty((B, Hq, n), dtype=torch.float32, device=dev)
                           for m in ("cross_full", "intra")}
-        if "lm_head" in kinds:
+        if kinds & {"lm_head", "lm_head_bwd"}:
             self.w_head = torch.empty((V, d), dtype=torch.bfloat16, device=dev).normal_(0, 3.0 / math.sqrt(d), generator=g)
             self.loss = torch.empty((B, L), dtype=torch.float32, device=dev)
             self.loss_lse = torch.empty((B, L), dtype=torch.float32, device=dev)
             self.ws_lm_n = hd.hd_lm_head_ce_workspace_bytes(B, L, V)
             self.ws_lm = torch.empty(self.ws_lm_n, dtype=torch.uint8, device=dev)
+        if "lm_head_bwd" in kinds:
+            self.dh = torch.empty((B, L, d), dtype=torch.bfloat16, device=dev)
+            self.dw_head = torch.empty((V, d), dtype=torch.float32, device=dev)
+            self.ws_lmb_n = hd.hd_lm_head_ce_bwd_workspace_bytes(B, L, V)
+            self.ws_lmb = torch.empty(self.ws_lmb_n, dtype=torch.uint8, device=dev)
         if "decode_final" in kinds:
             self.ws_fin_n = hd.hd_decode_final_workspace_bytes(B, n, T + 1, Hq, Hkv, D)
             self.ws_fin = torch.empty(self.ws_fin_n, dtype=torch.uint8, device=dev)
@@ -271,6 +281,9 @@ class Step:
         elif op["kind"] == "lm_head":
             hd.hd_lm_head_ce(d["x_hid"], self.w_head, d["labels"], self.loss, self.loss_lse, B, L, n,
                              wl["d"], wl["V"], self.ws_lm, self.ws_lm_n, s)
+        elif op["kind"] == "lm_head_bwd":
+            hd.hd_lm_head_ce_bwd(d["x_hid"], self.w_head, d["labels"], self.loss_lse, 1.0, self.dh,
+                                 self.dw_head, B, L, n, wl["d"], wl["V"], self.ws_lmb, self.ws_lmb_n, s)
         elif op["kind"] == "rope":
             hd.hd_rope_expanded(d["q"], d["k"], None, B, L, n, Hq, Hkv, D, 0, 10000.0, s)
         elif op["kind"] in ("fwd", "bwd"):
@@ -443,6 +456,8 @@ DESCRIPTIONS = {
                      "16384 prior tokens (65540 cache rows), Hq32 Hkv8 D128",
     "lm_head": "final-stream readout + fused LM-head cross-entropy, x [2,32768,4096] bf16 (16384 final-stream "
                "rows), head [32000,4096] bf16",
+    "lm_head_train": "final-stream LM-head cross-entropy and its gradients (dh, dW), x [2,32768,4096] bf16 "
+                     "(16384 final-stream rows), head [32000,4096] bf16",
     "rope": "RoPE in place at physical positions, q [1,131072,32,128] + k [1,131072,8,128] bf16, base 10000",
 }
 
@@ -622,7 +637,7 @@ def main():
         rec = {"ms": round(m, 4)}
         if op["flops"]:
             rec["tflops"] = round(op["flops"] / (m * 1e-3) / 1e12, 1)
-            if op["kind"] in ("fwd", "bwd", "lm_head"):
+            if op["kind"] in ("fwd", "bwd", "lm_head", "lm_head_bwd"):
                 rec["frac_of_measured_bf16"] = round(rec["tflops"] / tf_peak, 4)
         if op.get("bytes"):
             rec["gbs"] = round(op["bytes"] / (m * 1e-3) / 1e9, 1)
@@ -630,7 +645,7 @@ def main():
         per_op[op["name"]] = rec
     dom = max(ops, key=lambda o: per_op[o["name"]]["ms"])
     dom_ms = per_op[dom["name"]]["ms"]
-    if dom["kind"] in ("fwd", "bwd", "lm_head"):
+    if dom["kind"] in ("fwd", "bwd", "lm_head", "lm_head_bwd"):
         ach = dom["flops"] / (dom_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": tf_peak, "unit": "TFLOP/s",
                 "frac": round(ach / tf_peak, 4),
@@ -646,7 +661,8 @@ def main():
              "expand": "hd_expand_embed (expand_kernel)",
              "decode_final": "hd_decode_attn_final (decode_split + decode_combine)",
              "rope": "hd_rope_expanded (rope_kernel)",
-             "lm_head": "hd_lm_head_ce (lm_head_ce_kernel + lm_head_combine)"}[dom["kind"]]
+             "lm_head": "hd_lm_head_ce (lm_head_ce_kernel + lm_head_combine)",
+             "lm_head_bwd": "hd_lm_head_ce_bwd (gradient pass + two gemm_tc_kernel)"}[dom["kind"]]
     roof = {"kernel": f"{kname}, op {dom['name']}", **roof,
             "traffic": NCU_TRAFFIC.get((args.workload, dom["name"]))}
     if hbm_only:

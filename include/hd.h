@@ -155,6 +155,34 @@ int hd_lm_head_ce(const void* x, const void* w, const int32_t* labels, float* lo
                   int B, int L, int n, int d, int V, void* workspace, size_t workspace_bytes,
                   void* stream);
 
+/* Bytes of workspace hd_lm_head_ce_bwd needs (0 on invalid sizes). */
+size_t hd_lm_head_ce_bwd_workspace_bytes(int B, int L, int V);
+
+/*
+ * hd_lm_head_ce_bwd - gradients of the final-stream LM-head cross-entropy.
+ * Source: as hd_lm_head_ce (tahou.com page, "隐式序列缩放的技术细节" step 3).
+ *
+ * For the summed loss sum_r loss_r (tokens without a target contribute
+ * nothing), with G_r = softmax(h_r W^T) - onehot(labels[r]) (G_r = 0 when
+ * labels[r] < 0):
+ *
+ *   dh = grad_scale * G W      bf16 [B, L, d]: gradient w.r.t. the final-
+ *                              stream rows h (dX[b, t*n+n-1] = dh[b, t]; the
+ *                              other streams' rows of dX are zero)
+ *   dw = grad_scale * G^T h    fp32 [V, d]
+ *
+ *   x, w, labels  as hd_lm_head_ce; lse fp32 [B, L] from that call
+ *   grad_scale    e.g. 1 / (number of supervised tokens) for a mean loss
+ * G is recomputed from x and w (its logits on the tensor cores, fp32) and
+ * stored once as bf16 in the workspace; the two products accumulate in fp32.
+ * Supported: d a multiple of 64. `workspace` must hold
+ * hd_lm_head_ce_bwd_workspace_bytes(B, L, V) bytes (B*L rows of G, V rounded
+ * up to 256 columns).
+ */
+int hd_lm_head_ce_bwd(const void* x, const void* w, const int32_t* labels, const float* lse,
+                      float grad_scale, void* dh, float* dw, int B, int L, int n, int d, int V,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
 /*
  * hd_attn_fwd - Stream-Factorized attention forward.
  * Source: tahou.com page, "规模化落地的工程优化" (intra / cross-stream bullets,

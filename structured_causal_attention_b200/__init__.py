@@ -45,6 +45,8 @@ from ._lib import (  # noqa: F401
     hd_expand_embed,
     hd_final_readout,
     hd_lm_head_ce,
+    hd_lm_head_ce_bwd,
+    hd_lm_head_ce_bwd_workspace_bytes,
     hd_lm_head_ce_workspace_bytes,
     hd_rope_expanded,
     hd_selftest_wait_timeout,
@@ -205,3 +207,21 @@ def lm_head_ce(x, w, labels, n, stream=None, workspace=None):
     hd_lm_head_ce(x, w, labels, loss, lse, B, L, n, d, V, workspace,
                   workspace.numel() * workspace.element_size(), stream)
     return loss, lse
+
+
+def lm_head_ce_bwd(x, w, labels, lse, n, grad_scale=1.0, stream=None, workspace=None):
+    """Gradients of sum(loss) * grad_scale: (dh bf16 [B, L, d], dw fp32 [V, d])."""
+    import torch
+
+    _need_cuda(x, w, labels, lse)
+    B, S, d = x.shape
+    L = S // n
+    V = w.shape[0]
+    dh = torch.empty((B, L, d), dtype=torch.bfloat16, device=x.device)
+    dw = torch.empty((V, d), dtype=torch.float32, device=x.device)
+    nbytes = hd_lm_head_ce_bwd_workspace_bytes(B, L, V)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
+    hd_lm_head_ce_bwd(x, w, labels, lse, grad_scale, dh, dw, B, L, n, d, V, workspace,
+                      workspace.numel() * workspace.element_size(), stream)
+    return dh, dw

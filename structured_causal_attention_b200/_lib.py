@@ -34,6 +34,8 @@ SIGNATURES = {
     "hd_final_readout": (_I, [_P, _P, _I, _I, _I, _I, _I, _P]),
     "hd_lm_head_ce_workspace_bytes": (_Z, [_I, _I, _I]),
     "hd_lm_head_ce": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]),
+    "hd_lm_head_ce_bwd_workspace_bytes": (_Z, [_I, _I, _I]),
+    "hd_lm_head_ce_bwd": (_I, [_P, _P, _P, _P, _F, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]),
     "hd_attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "hd_attn_bwd_workspace_bytes": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
     "hd_attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I,
@@ -128,6 +130,17 @@ def hd_lm_head_ce(x, w, labels, loss, lse, B, L, n, d, V, workspace, workspace_b
     return _check(lib().hd_lm_head_ce(ptr(x), ptr(w), ptr(labels), ptr(loss), ptr(lse), B, L, n, d,
                                       V, ptr(workspace), workspace_bytes, stream_handle(stream)),
                   "hd_lm_head_ce")
+
+
+def hd_lm_head_ce_bwd_workspace_bytes(B, L, V):
+    return int(lib().hd_lm_head_ce_bwd_workspace_bytes(B, L, V))
+
+
+def hd_lm_head_ce_bwd(x, w, labels, lse, grad_scale, dh, dw, B, L, n, d, V, workspace, workspace_bytes,
+                      stream=None):
+    return _check(lib().hd_lm_head_ce_bwd(ptr(x), ptr(w), ptr(labels), ptr(lse), float(grad_scale), ptr(dh),
+                                          ptr(dw), B, L, n, d, V, ptr(workspace), workspace_bytes,
+                                          stream_handle(stream)), "hd_lm_head_ce_bwd")
 
 
 def hd_attn_fwd(q, k, v, out, lse, B, L, n, Hq, Hkv, D, mode, W_tokens, final_only, scale,

@@ -306,6 +306,39 @@ int hd_lm_head_ce(const void* x, const void* w, const int32_t* labels, float* lo
   return from_cuda(launch_lm_head_ce(p, x, w, n, sms, static_cast<cudaStream_t>(stream)));
 }
 
+size_t hd_lm_head_ce_bwd_workspace_bytes(int B, int L, int V) {
+  if (B < 1 || L < 1 || V < 1) return 0;
+  return lm_head_grad_workspace_bytes(static_cast<long long>(B) * L, V);
+}
+
+int hd_lm_head_ce_bwd(const void* x, const void* w, const int32_t* labels, const float* lse,
+                      float grad_scale, void* dh, float* dw, int B, int L, int n, int d, int V,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  if (!x || !w || !labels || !lse || !dh || !dw || !workspace) return HD_ERR_INVALID_ARG;
+  if (B < 1 || L < 1 || n < 1 || d < 1 || V < 1) return HD_ERR_INVALID_ARG;
+  if (!std::isfinite(grad_scale)) return HD_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(dh) || !aligned16(dw) || !aligned16(workspace))
+    return HD_ERR_INVALID_ARG;
+  if (d % 64 != 0) return HD_ERR_UNSUPPORTED;
+  const long long R = static_cast<long long>(B) * L;
+  if (R > (1LL << 31) - 1) return HD_ERR_UNSUPPORTED;
+  if (workspace_bytes < lm_head_grad_workspace_bytes(R, V)) return HD_ERR_INVALID_ARG;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+    return HD_ERR_CUDA;
+  LmHeadParams p{};
+  p.labels = labels;
+  p.lse_in = lse;
+  p.g = static_cast<__nv_bfloat16*>(workspace);
+  p.R = R;
+  p.V = V;
+  p.d = d;
+  p.status = status_ptr();
+  return from_cuda(launch_lm_head_ce_bwd(p, x, w, n, grad_scale, dh, dw, sms,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
 int hd_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int L,
                 int n, int Hq, int Hkv, int D, int mode, int W_tokens,
                 int final_stream_queries_only, float scale, void* stream) {

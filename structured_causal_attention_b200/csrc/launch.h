@@ -62,8 +62,15 @@ struct LmHeadParams {
   int V, d;
   int nrb, nvt;           // row pairs, vocabulary tiles (set by the launcher)
   long long units;
+  // gradient pass only
+  const float* lse_in;    // [R] natural-log LSE of the forward
+  __nv_bfloat16* g;       // [R, g_ld] softmax - onehot, bf16
+  long long g_ld;         // columns of g: V rounded up to 256
 };
 size_t lm_head_workspace_bytes(long long R, int V);
+size_t lm_head_grad_workspace_bytes(long long R, int V);
+cudaError_t launch_lm_head_ce_bwd(LmHeadParams p, const void* x, const void* w, int n, float scale,
+                                  void* dh, float* dw, int num_sms, cudaStream_t stream);
 cudaError_t launch_lm_head_ce(LmHeadParams p, const void* x, const void* w, int n, int num_sms,
                               cudaStream_t stream);
 cudaError_t launch_final_readout(const void* x, void* out, long long rows, int n,

@@ -84,6 +84,11 @@ __device__ __forceinline__ float select32(const uint32_t* x, int k) {
   return __uint_as_float((k & 1) ? v[1] : v[0]);
 }
 
+// kGrad = false: the loss epilogue (per-tile max / sum of exp2, label logit).
+// kGrad = true: the gradient epilogue, G[r, v] = 2^(logit log2 e - LSE_r log2 e)
+// - [v == label_r] as bf16 into p.g (row stride p.g_ld), zero for rows without
+// a target and for the padding columns v >= V.
+template <bool kGrad>
 __global__ void __launch_bounds__(kLThreads, 1)
     lm_head_ce_kernel(const LmHeadParams p, const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmW) {
@@ -177,37 +182,72 @@ __global__ void __launch_bounds__(kLThreads, 1)
         row[h] = w.rb * 2 * kLR + h * kLR + quarter * 32 + lane;
         lab[h] = row[h] < p.R ? __ldg(p.labels + row[h]) : -1;
       }
+      float lse2[2];
+      if constexpr (kGrad) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) lse2[h] = row[h] < p.R ? __ldg(p.lse_in + row[h]) * kLog2e : 0.f;
+      }
       if (!tc::mbar_wait(bar(LB_ACC_FULL), ui & 1, abort_flag, p.status)) break;
       tc::tc_fence_after();
-      const int nchunk = min(kLV, p.V - v0 + 31) / 32;  // chunks with at least one entry < V
+      if constexpr (kGrad) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float m = -INFINITY, l = 0.f, picked = 0.f;
-        const int lo = lab[h] - v0;  // label's column in this tile, if in [0, 256)
-        for (int c = 0; c < nchunk; ++c) {
-          uint32_t x[32];
-          tc::tmem_ld32(tq + h * kLV + c * 32, x);
-          tc::tmem_wait_ld();
-          if (lo >= c * 32 && lo < c * 32 + 32) picked = select32(x, lo - c * 32);
-          const int valid = min(32, p.V - (v0 + c * 32));  // >= 1
-          float y[32];
-          float mx = -INFINITY;
+        for (int h = 0; h < 2; ++h) {
+          const bool live = row[h] < p.R && lab[h] >= 0 && lab[h] < p.V;
+          __nv_bfloat16* grow = p.g + static_cast<long long>(row[h]) * p.g_ld + v0;
+          for (int c = 0; c < kLV / 32; ++c) {
+            uint32_t x[32];
+            tc::tmem_ld32(tq + h * kLV + c * 32, x);
+            tc::tmem_wait_ld();
+            uint32_t pk[16];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            y[j] = j < valid ? __uint_as_float(x[j]) * kLog2e : -INFINITY;
-            mx = fmaxf(mx, y[j]);
+            for (int j = 0; j < 32; j += 2) {
+              const int v = v0 + c * 32 + j;
+              float g0 = fast_exp2(fmaf(__uint_as_float(x[j]), kLog2e, -lse2[h])) - (v == lab[h] ? 1.f : 0.f);
+              float g1 = fast_exp2(fmaf(__uint_as_float(x[j + 1]), kLog2e, -lse2[h])) -
+                         (v + 1 == lab[h] ? 1.f : 0.f);
+              g0 = (live && v < p.V) ? g0 : 0.f;
+              g1 = (live && v + 1 < p.V) ? g1 : 0.f;
+              pk[j >> 1] = pack_bf16(g0, g1);
+            }
+            if (row[h] < p.R) {
+              uint4* dst = reinterpret_cast<uint4*>(grow + c * 32);
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4)
+                dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+            }
           }
-          const float mn = fmaxf(m, mx);
-          float s = 0.f;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) s += fast_exp2(y[j] - mn);
-          l = l * fast_exp2(m - mn) + s;
-          m = mn;
         }
-        if (row[h] < p.R) {
-          p.part[static_cast<long long>(w.vt) * p.R + row[h]] = m;
-          p.part[static_cast<long long>(p.nvt + w.vt) * p.R + row[h]] = l;
-          if (lo >= 0 && lo < kLV) p.pick[row[h]] = picked;
+      } else {
+        const int nchunk = min(kLV, p.V - v0 + 31) / 32;  // chunks with at least one entry < V
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float m = -INFINITY, l = 0.f, picked = 0.f;
+          const int lo = lab[h] - v0;  // label's column in this tile, if in [0, 256)
+          for (int c = 0; c < nchunk; ++c) {
+            uint32_t x[32];
+            tc::tmem_ld32(tq + h * kLV + c * 32, x);
+            tc::tmem_wait_ld();
+            if (lo >= c * 32 && lo < c * 32 + 32) picked = select32(x, lo - c * 32);
+            const int valid = min(32, p.V - (v0 + c * 32));  // >= 1
+            float y[32];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              y[j] = j < valid ? __uint_as_float(x[j]) * kLog2e : -INFINITY;
+              mx = fmaxf(mx, y[j]);
+            }
+            const float mn = fmaxf(m, mx);
+            float s = 0.f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) s += fast_exp2(y[j] - mn);
+            l = l * fast_exp2(m - mn) + s;
+            m = mn;
+          }
+          if (row[h] < p.R) {
+            p.part[static_cast<long long>(w.vt) * p.R + row[h]] = m;
+            p.part[static_cast<long long>(p.nvt + w.vt) * p.R + row[h]] = l;
+            if (lo >= 0 && lo < kLV) p.pick[row[h]] = picked;
+          }
         }
       }
       tc::tc_fence_before();
@@ -220,6 +260,169 @@ __global__ void __launch_bounds__(kLThreads, 1)
   if (warp == 1) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, kLTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// C[M, N] = scale * A[M, K] B[K, N] on the tensor cores (bf16 operands, fp32
+// accumulation in TMEM): the two GEMMs of the LM-head gradient. Persistent;
+// a unit is one 128 x 256 tile of C, units walked with the N tiles inner so
+// the CTAs running at once share their A rows in L2.
+//   A: K-major (row m of A contiguous) or, with kAmn, M-major (A stored as
+//      A^T, i.e. row k contiguous over m). B: N-major (row k contiguous).
+//   warp 0    TMA producer, 64-wide K blocks into a 4-stage ring
+//   warp 1    TMEM (2 accumulators of 256 columns); lane 0 issues M128 N256
+//             K16 MMAs (long enough that issue keeps up with the tensor cores)
+//   warps 2-5 epilogue: a row per thread, tcgen05.ld, scale, 16-byte stores;
+//             the other accumulator takes the next unit's MMAs meanwhile.
+constexpr int kGM = 128, kGN = 256, kGK = 64, kGStages = 4, kGThreads = 192;
+constexpr int kGABytes = kGM * kGK * 2;   // 16 KB
+constexpr int kGBBytes = kGK * kGN * 2;   // 32 KB
+constexpr int kGStageBytes = kGABytes + kGBBytes;
+enum { GB_FULL = 0, GB_EMPTY = kGStages, GB_AF = 2 * kGStages, GB_AE = GB_AF + 2, GB_N = GB_AE + 2 };
+constexpr int kGBarOff = kGStages * kGStageBytes;
+constexpr int kGSlotOff = kGBarOff + GB_N * 8;
+constexpr int kGAbortOff = kGSlotOff + 4;
+constexpr int kGSmem = kGAbortOff + 4 + 1024;
+static_assert(kGSmem <= 232448, "shared memory");
+
+struct GemmArgs {
+  void* c;         // [M, ldc] bf16, or fp32 when c_fp32
+  long long ldc;
+  int M, N, K, c_fp32;
+  float scale;
+  int ntn;         // N tiles
+  long long units;
+  int* status;
+};
+
+template <bool kAmn>
+__global__ void __launch_bounds__(kGThreads, 1)
+    gemm_tc_kernel(const GemmArgs p, const __grid_constant__ CUtensorMap tmA,
+                   const __grid_constant__ CUtensorMap tmB) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
+  auto bar = [&](int i) { return sbase + kGBarOff + 8u * i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + kGAbortOff);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (p.status && *reinterpret_cast<volatile int*>(p.status) == HD_ERR_TIMEOUT) return;
+  if (tid == 0) {
+    for (int i = 0; i < GB_N; ++i) tc::mbar_init(bar(i), (i == GB_AE || i == GB_AE + 1) ? 4 : 1);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(sbase + kGSlotOff, 512);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sgen + kGSlotOff);
+  const int nkb = (p.K + kGK - 1) / kGK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tc::tma_prefetch_desc(&tmA);
+      tc::tma_prefetch_desc(&tmB);
+      int it = 0;
+      bool ok = true;
+      for (long long u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+        const int m0 = static_cast<int>(u / p.ntn) * kGM, n0 = static_cast<int>(u % p.ntn) * kGN;
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % kGStages;
+          if (!tc::mbar_wait(bar(GB_EMPTY + s), ((it / kGStages) & 1) ^ 1, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = sbase + s * kGStageBytes, sb = sa + kGABytes;
+          tc::mbar_expect_tx(bar(GB_FULL + s), kGStageBytes);
+          if (kAmn) {
+            tc::tma_load_2d(sa, &tmA, bar(GB_FULL + s), m0, kb * kGK);
+            tc::tma_load_2d(sa + kGABytes / 2, &tmA, bar(GB_FULL + s), m0 + 64, kb * kGK);
+          } else {
+            tc::tma_load_2d(sa, &tmA, bar(GB_FULL + s), kb * kGK, m0);
+          }
+#pragma unroll
+          for (int q4 = 0; q4 < kGN / 64; ++q4)
+            tc::tma_load_2d(sb + q4 * (kGBBytes / 4), &tmB, bar(GB_FULL + s), n0 + 64 * q4, kb * kGK);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = tc::idesc_bf16_f32(kGM, kGN, kAmn ? 1 : 0, 1);
+      int it = 0, ui = 0;
+      bool ok = true;
+      for (long long u = blockIdx.x; ok && u < p.units; u += gridDim.x, ++ui) {
+        const int buf = ui & 1;
+        // the epilogue has read this accumulator's previous unit
+        if (ui >= 2 && !tc::mbar_wait(bar(GB_AE + buf), ((ui >> 1) - 1) & 1, abort_flag, p.status)) break;
+        tc::tc_fence_after();
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % kGStages;
+          if (!tc::mbar_wait(bar(GB_FULL + s), (it / kGStages) & 1, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc::tc_fence_after();
+          const uint32_t sa = sbase + s * kGStageBytes, sb = sa + kGABytes;
+#pragma unroll
+          for (int kk = 0; kk < kGK / 16; ++kk) {
+            const uint64_t ad = kAmn ? tc::smem_desc_sw128(sa + kk * 2048, kGABytes / 2, 1024)
+                                     : tc::smem_desc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t bd = tc::smem_desc_sw128(sb + kk * 2048, kGBBytes / 4, 1024);
+            tc::mma_ss(tmem + kGN * buf, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc::mma_commit(bar(GB_EMPTY + s));
+        }
+        if (ok) tc::mma_commit(bar(GB_AF + buf));
+      }
+    }
+  } else {
+    const int quarter = warp & 3;
+    const uint32_t tq = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    int ui = 0;
+    for (long long u = blockIdx.x; u < p.units; u += gridDim.x, ++ui) {
+      const int buf = ui & 1;
+      const int m0 = static_cast<int>(u / p.ntn) * kGM, n0 = static_cast<int>(u % p.ntn) * kGN;
+      const int r = m0 + quarter * 32 + lane;
+      if (!tc::mbar_wait(bar(GB_AF + buf), (ui >> 1) & 1, abort_flag, p.status)) break;
+      tc::tc_fence_after();
+      for (int c = 0; c < kGN / 32; ++c) {
+        uint32_t x[32];
+        tc::tmem_ld32(tq + kGN * buf + c * 32, x);
+        tc::tmem_wait_ld();
+        const int col = n0 + c * 32;
+        if (r < p.M && col < p.N) {
+          if (p.c_fp32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.c) + r * p.ldc + col);
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4)
+              dst[q4] = make_float4(__uint_as_float(x[4 * q4]) * p.scale, __uint_as_float(x[4 * q4 + 1]) * p.scale,
+                                    __uint_as_float(x[4 * q4 + 2]) * p.scale, __uint_as_float(x[4 * q4 + 3]) * p.scale);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.c) + r * p.ldc + col);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const float* f = reinterpret_cast<const float*>(x + 8 * q4);
+              dst[q4] = make_uint4(pack_bf16(f[0] * p.scale, f[1] * p.scale), pack_bf16(f[2] * p.scale, f[3] * p.scale),
+                                   pack_bf16(f[4] * p.scale, f[5] * p.scale), pack_bf16(f[6] * p.scale, f[7] * p.scale));
+            }
+          }
+        }
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar(GB_AE + buf));
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 512);
   }
 }
 
@@ -314,15 +517,95 @@ cudaError_t launch_lm_head_ce(LmHeadParams p, const void* x, const void* w, int 
   p.nrb = static_cast<int>((p.R + 2 * kLR - 1) / (2 * kLR));
   p.nvt = (p.V + kLV - 1) / kLV;
   p.units = static_cast<long long>(p.nrb) * p.nvt;
-  cudaError_t e = cudaFuncSetAttribute(lm_head_ce_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kLSmem);
+  cudaError_t e = cudaFuncSetAttribute(lm_head_ce_kernel<false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kLSmem);
   if (e != cudaSuccess) return e;
   const long long grid = p.units < num_sms ? p.units : num_sms;
-  lm_head_ce_kernel<<<static_cast<unsigned>(grid), kLThreads, kLSmem, stream>>>(p, ma, mw);
+  lm_head_ce_kernel<false><<<static_cast<unsigned>(grid), kLThreads, kLSmem, stream>>>(p, ma, mw);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   lm_head_combine_kernel<<<static_cast<unsigned>((p.R + 255) / 256), 256, 0, stream>>>(p);
   return cudaGetLastError();
+}
+
+size_t lm_head_grad_workspace_bytes(long long R, int V) {
+  const long long vp = (V + kLV - 1) / kLV * kLV;
+  return (static_cast<size_t>(R * vp) * 2 + 255) & ~static_cast<size_t>(255);
+}
+
+namespace {
+
+template <bool kAmn>
+cudaError_t launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, GemmArgs a, int num_sms,
+                        cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<kAmn>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kGSmem);
+  if (e != cudaSuccess) return e;
+  const long long grid = a.units < num_sms ? a.units : num_sms;
+  gemm_tc_kernel<kAmn><<<static_cast<unsigned>(grid), kGThreads, kGSmem, stream>>>(a, ma, mb);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_lm_head_ce_bwd(LmHeadParams p, const void* x, const void* w, int n, float scale,
+                                  void* dh, float* dw, int num_sms, cudaStream_t stream) {
+  const __nv_bfloat16* h_base = static_cast<const __nv_bfloat16*>(x) + static_cast<long long>(n - 1) * p.d;
+  const long long hstride = static_cast<long long>(n) * p.d;
+  // 1. G = softmax(logits) - onehot, bf16 [R, g_ld]
+  CUtensorMap ma, mw;
+  if (!make_map_2d(&ma, h_base, p.d, p.R, hstride, kLR) || !make_map_2d(&mw, w, p.d, p.V, p.d, kLV))
+    return cudaErrorInvalidValue;
+  p.nrb = static_cast<int>((p.R + 2 * kLR - 1) / (2 * kLR));
+  p.nvt = (p.V + kLV - 1) / kLV;
+  p.units = static_cast<long long>(p.nrb) * p.nvt;
+  p.g_ld = static_cast<long long>(p.nvt) * kLV;
+  cudaError_t e = cudaFuncSetAttribute(lm_head_ce_kernel<true>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kLSmem);
+  if (e != cudaSuccess) return e;
+  long long grid = p.units < num_sms ? p.units : num_sms;
+  lm_head_ce_kernel<true><<<static_cast<unsigned>(grid), kLThreads, kLSmem, stream>>>(p, ma, mw);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int ntn = (p.d + kGN - 1) / kGN;
+  // 2. dh = scale * G W: A = G (K-major over the vocabulary), B = W (rows = vocabulary)
+  {
+    CUtensorMap ga, gb;
+    if (!make_map_2d(&ga, p.g, p.g_ld, p.R, p.g_ld, kGM) || !make_map_2d(&gb, w, p.d, p.V, p.d, kGK))
+      return cudaErrorInvalidValue;
+    GemmArgs a{};
+    a.c = dh;
+    a.ldc = p.d;
+    a.M = static_cast<int>(p.R);
+    a.N = p.d;
+    a.K = static_cast<int>(p.g_ld);
+    a.c_fp32 = 0;
+    a.scale = scale;
+    a.ntn = ntn;
+    a.units = (p.R + kGM - 1) / kGM * ntn;
+    a.status = p.status;
+    e = launch_gemm<false>(ga, gb, a, num_sms, stream);
+    if (e != cudaSuccess) return e;
+  }
+  // 3. dW = scale * G^T h: A = G read vocabulary-major, B = the final-stream rows in place
+  {
+    CUtensorMap ga, gb;
+    if (!make_map_2d(&ga, p.g, p.g_ld, p.R, p.g_ld, kGK) || !make_map_2d(&gb, h_base, p.d, p.R, hstride, kGK))
+      return cudaErrorInvalidValue;
+    GemmArgs a{};
+    a.c = dw;
+    a.ldc = p.d;
+    a.M = p.V;
+    a.N = p.d;
+    a.K = static_cast<int>(p.R);
+    a.c_fp32 = 1;
+    a.scale = scale;
+    a.ntn = ntn;
+    a.units = static_cast<long long>((p.V + kGM - 1) / kGM) * ntn;
+    a.status = p.status;
+    e = launch_gemm<true>(ga, gb, a, num_sms, stream);
+  }
+  return e;
 }
 
 cudaError_t launch_final_readout(const void* x, void* out, long long rows, int n,

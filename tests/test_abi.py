@@ -138,6 +138,21 @@ def test_lm_head_workspace_and_rejects(lib):
     assert L.hd_final_readout(0, FAKE, 1, 4, 2, 8, 2, None) == hd.HD_ERR_INVALID_ARG
 
 
+def test_lm_head_bwd_workspace_and_rejects(lib):
+    L = hd.lib()
+    ws = hd.hd_lm_head_ce_bwd_workspace_bytes(2, 100, 1000)
+    assert ws == 200 * 1024 * 2  # B*L rows of G, V rounded up to 256 columns, bf16
+    ok = [FAKE, FAKE, FAKE, FAKE, 1.0, FAKE, FAKE, 2, 100, 4, 128, 1000, FAKE, ws, None]
+    bad = list(ok); bad[12 + 1] = ws - 1
+    assert L.hd_lm_head_ce_bwd(*bad) == hd.HD_ERR_INVALID_ARG
+    bad = list(ok); bad[10] = 96
+    assert L.hd_lm_head_ce_bwd(*bad) == hd.HD_ERR_UNSUPPORTED
+    bad = list(ok); bad[4] = float("nan")
+    assert L.hd_lm_head_ce_bwd(*bad) == hd.HD_ERR_INVALID_ARG
+    bad = list(ok); bad[3] = 0
+    assert L.hd_lm_head_ce_bwd(*bad) == hd.HD_ERR_INVALID_ARG
+
+
 def test_expand_rejects(lib):
     L = hd.lib()
     assert L.hd_expand_embed(FAKE, FAKE, FAKE, 1, 4, 2, 0, 8, 4, None) == hd.HD_ERR_INVALID_ARG

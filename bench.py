@@ -14,6 +14,12 @@ expanded positions, 16 query / 4 KV heads, head_dim 128):
 value = unmasked attention TFLOP/s over the step (fwd 4*D, bwd 10*D FLOPs per
 visible (query, key, head) pair, decode 4*D per pair).
 
+--workload selects a single-configuration measurement instead: intra_train,
+cross_window, long_cross (fwd/bwd at those sizes), decode8 / decode64 /
+decode8_final (decode steps), expand, rope (RoPE of q and k at 131072
+positions), lm_head and lm_head_train (final-stream LM-head cross-entropy, and
+with its gradients). HBM-bound workloads report GB/s, the rest TFLOP/s.
+
 --impl reference times the float64 CPU oracle (the reference arm) on a bounded
 sample of the same workload. Multi-GPU (torchrun): every rank runs its own
 replica of the step (data parallel, no collective on the data path).

@@ -37,9 +37,10 @@
  *     stream). Every call only enqueues work on that stream and returns.
  *   - Argument errors are reported (HD_ERR_INVALID_ARG / HD_ERR_UNSUPPORTED)
  *     before anything is launched. A failed launch returns HD_ERR_CUDA.
- *     Errors found on the device (a token id outside the table, a bounded
- *     wait that gave up) are recorded in a per-device status word, read and
- *     cleared with hd_device_status(); kernels never trap.
+ *     Errors found on the device (a token id, label, sequence length or token
+ *     offset out of range, a bounded wait that gave up) are recorded in a
+ *     per-device status word, read and cleared with hd_device_status();
+ *     kernels never trap.
  */
 #ifndef HD_H_
 #define HD_H_
@@ -65,7 +66,9 @@ typedef enum { HD_INTRA = 0, HD_CROSS_FULL = 1, HD_CROSS_WINDOW = 2 } hd_mode;
 /* Human-readable name of a status code (static string, never NULL). */
 const char* hd_status_string(int status);
 
-/* Library ABI version: (major << 16) | minor. */
+/* Library ABI version: (major << 16) | minor. Minor 1 added RoPE, the
+ * final-stream readout, the LM-head cross-entropy and its gradients,
+ * final-stream-only decode and the bounded-wait self-test. */
 int hd_version(void);
 
 /*

@@ -217,7 +217,7 @@ const char* hd_status_string(int status) {
   }
 }
 
-int hd_version(void) { return (1 << 16) | 0; }
+int hd_version(void) { return (1 << 16) | 1; }
 
 int hd_expand_embed(const int32_t* ids, const void* tables, void* out, int B, int L, int n, int V,
                     int d, int elem_bytes, void* stream) {

@@ -24,11 +24,12 @@
 //               bulk reduce-add (the TMA unit does the adds, not the SM).
 //   warp 12     TMA: K, V once; Q and dO tiles (3 stages) plus the tile's
 //               packed LSE and D rows (bulk copies).
-//   warp 13     TMEM allocation; lane 0 issues dV, dK and dQ^T.
-//   warp 14     lane 0 issues S^T and dP^T of the next tile.
-// One thread issues a tcgen05.mma only every ~75 cycles, more than twice what
-// an N=64 MMA takes to run, so the two groups get an issuer each; their
-// hand-offs go through the barriers below, not through issue order.
+//   warp 13     TMEM allocation; issues dV, dK and dQ^T.
+//   warp 14     issues S^T and dP^T of the next tile.
+// Each issuer warp walks its loop as a whole warp (warp-uniform operands) and
+// one elected lane issues. The two groups wait on different barriers (P^T
+// written vs. the next stage loaded and its buffer free), so each has its own
+// warp; their hand-offs go through the barriers below, not issue order.
 // Every mbarrier wait is bounded (HD_ERR_TIMEOUT, then every role leaves).
 #include <cuda.h>
 
@@ -184,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 13 || warp == 14) {
     // ------------------------------------------------------------ MMA issuers
-    if (lane == 0 && total > 0) {
+    if (total > 0) {  // the whole warp walks the issue loop; one elected lane issues
       constexpr uint32_t idSP = tc::idesc_bf16_f32(128, kQM, 0, 0);  // S^T, dP^T
       constexpr uint32_t idKV = tc::idesc_bf16_f32(128, D, 0, 1);    // dV, dK
       constexpr uint32_t idDQ = tc::idesc_bf16_f32(128, kQM, 1, 1);  // dQ^T
@@ -199,32 +200,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dSm = tc::smem_desc_sw128(sDS, SM::QSUB, 1024);
       const uint64_t dKt = tc::smem_desc_sw128(sK, kt_lbo, 1024);
       auto add = [](uint64_t d, uint32_t bytes) { return d + (bytes >> 4); };
-      bool ok = tc::mbar_wait(bar(B_KV), 0, abort_flag, p.status);
+      bool ok = tc::mbar_wait_warp(bar(B_KV), 0, abort_flag, p.status);
       if (warp == 14) {
         // S^T, dP^T of tile it into TMEM buffer it & 1, once the stage is
         // loaded and dQ^T of tile it-2 (same buffer) has been read out
         for (int it = 0; ok && it < total; ++it) {
           const int x = it & 1, st = it % kQS;
-          ok = tc::mbar_wait(bar(B_QF + st), (it / kQS) & 1, abort_flag, p.status);
-          if (ok && it >= 2) ok = tc::mbar_wait(bar(B_DE + x), ((it >> 1) - 1) & 1, abort_flag, p.status);
+          ok = tc::mbar_wait_warp(bar(B_QF + st), (it / kQS) & 1, abort_flag, p.status);
+          if (ok && it >= 2) ok = tc::mbar_wait_warp(bar(B_DE + x), ((it >> 1) - 1) & 1, abort_flag, p.status);
           if (!ok) break;
           tc::tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t ko = (kk >> 2) * SM::KSUB + (kk & 3) * 32;
             const uint32_t qo = (st * NSUB + (kk >> 2)) * SM::QSUB + (kk & 3) * 32;
-            tc::mma_ss(tmem + 128 * x, add(dK, ko), add(dQk, qo), idSP, kk > 0);
-            tc::mma_ss(tmem + 128 * x + 64, add(dV, ko), add(dOk, qo), idSP, kk > 0);
+            tc::mma_ss_elect(tmem + 128 * x, add(dK, ko), add(dQk, qo), idSP, kk > 0);
+            tc::mma_ss_elect(tmem + 128 * x + 64, add(dV, ko), add(dOk, qo), idSP, kk > 0);
           }
-          tc::mma_commit(bar(B_SF + x));
-          tc::mma_commit(bar(B_QE + st));
+          tc::mma_commit_elect(bar(B_SF + x));
+          tc::mma_commit_elect(bar(B_QE + st));
         }
       } else {
         // dV, dK, dQ^T of tile it once P^T / dS^T are written
         for (int it = 0; ok && it < total; ++it) {
           const int x = it & 1, st = it % kQS;
-          ok = tc::mbar_wait(bar(B_QF + st), (it / kQS) & 1, abort_flag, p.status) &&
-               tc::mbar_wait(bar(B_PF), it & 1, abort_flag, p.status);
+          ok = tc::mbar_wait_warp(bar(B_QF + st), (it / kQS) & 1, abort_flag, p.status) &&
+               tc::mbar_wait_warp(bar(B_PF), it & 1, abort_flag, p.status);
           if (!ok) break;
           tc::tc_fence_after();
           const uint32_t acc = it > 0 ? 1u : 0u;
@@ -234,22 +235,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t as = add(dS, kk * 32);
             const uint64_t bo = add(dOm, st * NSUB * SM::QSUB + kk * 2048);
             const uint64_t bq = add(dQm, st * NSUB * SM::QSUB + kk * 2048);
-            tc::mma_ss(tdV, ap, bo, idKV, (acc | kk) ? 1u : 0u);
-            tc::mma_ss(tdK, as, bq, idKV, (acc | kk) ? 1u : 0u);
+            tc::mma_ss_elect(tdV, ap, bo, idKV, (acc | kk) ? 1u : 0u);
+            tc::mma_ss_elect(tdK, as, bq, idKV, (acc | kk) ? 1u : 0u);
           }
 #pragma unroll
           for (int kk = 0; kk < kKN / 16; ++kk) {  // reduce over the 128 keys
             const uint64_t ak = add(dKt, kk * 2048);
             const uint64_t bs = add(dSm, kk * 2048);
-            tc::mma_ss(tmem + 128 * x, ak, bs, idDQ, kk > 0 ? 1u : 0u);
+            tc::mma_ss_elect(tmem + 128 * x, ak, bs, idDQ, kk > 0 ? 1u : 0u);
           }
-          tc::mma_commit(bar(B_DF + x));
-          tc::mma_commit(bar(B_QE + st));
-          tc::mma_commit(bar(B_PE));
+          tc::mma_commit_elect(bar(B_DF + x));
+          tc::mma_commit_elect(bar(B_QE + st));
+          tc::mma_commit_elect(bar(B_PE));
         }
         // every S^T / dP^T MMA finished before the last P^T was written, so this
         // covers both issuers
-        tc::mma_commit(bar(B_END));
+        tc::mma_commit_elect(bar(B_END));
       }
     }
   } else if (warp < 8) {

@@ -16,13 +16,15 @@
 //               upper S columns of TMEM (tcgen05.st). The running max is only raised
 //               when a tile's max exceeds it by more than 2^8, so the O
 //               accumulator is rescaled in TMEM rarely; the final 1/l and LSE
-//               make the result exact either way.
+//               make the result exact either way. The reload of keys 0-63 is
+//               issued while keys 64-127 are still being exponentiated.
 //   warp 8      TMA producer: both Q tiles once, then K and V tiles of 128 keys
 //               into a 2-stage ring (128-byte swizzle). The 4-D tensor maps are
 //               (d, head-or-stream*head, row, batch), so an INTRA stream is read
 //               as a contiguous causal problem (row stride n*H*D), with no copy.
-//   warp 9      allocates TMEM (2 x [S/P 128 columns | O D columns]); lane 0
-//               issues every tcgen05.mma in the order
+//   warp 9      allocates TMEM (2 x [S/P 128 columns | O D columns]) and walks
+//               the MMA loop as a whole warp (warp-uniform operands), one
+//               elected lane issuing every tcgen05.mma, in the order
 //                   PV_0(j), S_0(j+1), PV_1(j), S_1(j+1)
 //               so one tile's MMAs run while the other tile's softmax works.
 //               S = Q K^T (M=128, N=128, both operands from shared memory);
@@ -170,21 +172,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    {  // the whole warp walks the issue loop; one elected lane issues
       constexpr uint32_t idS = tc::idesc_bf16_f32(kBM, kBN, 0, 0);
       constexpr uint32_t idO = tc::idesc_bf16_f32(kBM, D, 0, 1);
       auto issue_S = [&](int q, int st) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
-          tc::mma_ss(tmem + 256 * q, tc::smem_desc_sw128(sQ + q * SM::Q_BYTES + off, 16, 1024),
-                     tc::smem_desc_sw128(sK + st * SM::KV_BYTES + off, 16, 1024), idS, kk > 0);
+          tc::mma_ss_elect(tmem + 256 * q, tc::smem_desc_sw128(sQ + q * SM::Q_BYTES + off, 16, 1024),
+                           tc::smem_desc_sw128(sK + st * SM::KV_BYTES + off, 16, 1024), idS, kk > 0);
         }
-        tc::mma_commit(bar(B_SF + q));
+        tc::mma_commit_elect(bar(B_SF + q));
       };
       int pf_count[2] = {0, 0};
-      bool ok = tc::mbar_wait(bar(B_QF), 0, abort_flag, p.status) &&
-                tc::mbar_wait(bar(B_KF), 0, abort_flag, p.status);
+      bool ok = tc::mbar_wait_warp(bar(B_QF), 0, abort_flag, p.status) &&
+                tc::mbar_wait_warp(bar(B_KF), 0, abort_flag, p.status);
       if (ok) {
         tc::tc_fence_after();
 #pragma unroll
@@ -199,29 +201,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (in_range(q, j)) {
             // PV in two halves of 64 keys: keys 64-127 as soon as their P is
             // written, while the softmax still works on keys 0-63
-            ok = tc::mbar_wait(bar(B_PA + q), pf_count[q] & 1, abort_flag, p.status);
-            if (ok && !v_ready) ok = tc::mbar_wait(bar(B_VF + st), (i >> 1) & 1, abort_flag, p.status);
+            ok = tc::mbar_wait_warp(bar(B_PA + q), pf_count[q] & 1, abort_flag, p.status);
+            if (ok && !v_ready) ok = tc::mbar_wait_warp(bar(B_VF + st), (i >> 1) & 1, abort_flag, p.status);
             if (!ok) break;
             v_ready = true;
             tc::tc_fence_after();
 #pragma unroll
             for (int kk = kBN / 32; kk < kBN / 16; ++kk)
-              tc::mma_ts(tmem + 256 * q + 128, tmem + 256 * q + 64 + kk * 8,
-                         tc::smem_desc_sw128(sV + st * SM::KV_BYTES + kk * 2048, kSub, 1024), idO,
-                         (j > lo[q] || kk > kBN / 32) ? 1u : 0u);
-            ok = tc::mbar_wait(bar(B_PB + q), pf_count[q] & 1, abort_flag, p.status);
+              tc::mma_ts_elect(tmem + 256 * q + 128, tmem + 256 * q + 64 + kk * 8,
+                               tc::smem_desc_sw128(sV + st * SM::KV_BYTES + kk * 2048, kSub, 1024), idO,
+                               (j > lo[q] || kk > kBN / 32) ? 1u : 0u);
+            ok = tc::mbar_wait_warp(bar(B_PB + q), pf_count[q] & 1, abort_flag, p.status);
             if (!ok) break;
             ++pf_count[q];
             tc::tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < kBN / 32; ++kk)
-              tc::mma_ts(tmem + 256 * q + 128, tmem + 256 * q + 64 + kk * 8,
-                         tc::smem_desc_sw128(sV + st * SM::KV_BYTES + kk * 2048, kSub, 1024), idO, 1u);
-            if (j == hi[q]) tc::mma_commit(bar(B_OF + q));
+              tc::mma_ts_elect(tmem + 256 * q + 128, tmem + 256 * q + 64 + kk * 8,
+                               tc::smem_desc_sw128(sV + st * SM::KV_BYTES + kk * 2048, kSub, 1024), idO, 1u);
+            if (j == hi[q]) tc::mma_commit_elect(bar(B_OF + q));
           }
           if (in_range(q, j + 1)) {
             if (!k_next_ready) {
-              ok = tc::mbar_wait(bar(B_KF + s1), ((i + 1) >> 1) & 1, abort_flag, p.status);
+              ok = tc::mbar_wait_warp(bar(B_KF + s1), ((i + 1) >> 1) & 1, abort_flag, p.status);
               if (!ok) break;
               k_next_ready = true;
               tc::tc_fence_after();
@@ -229,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             issue_S(q, s1);
           }
         }
-        tc::mma_commit(bar(B_KE + st));
+        tc::mma_commit_elect(bar(B_KE + st));
       }
     }
   } else {
@@ -253,50 +255,57 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int c0 = j * kBN;
       const bool full = (c0 + kBN - 1 <= p.a * rq0 + p.bb) &&
                         (c0 > p.a * rq_last + p.bb - p.win) && (c0 + kBN <= p.Lk);
-      // Three TMEM round trips per tile with at most 64 scores live: keys 0-63
-      // (max), keys 64-127 (max, then their P), keys 0-63 again (their P).
+      // The row's 128 scores are read from TMEM once for the max; keys 64-127
+      // stay in registers for their P, and keys 0-63 are read again, those
+      // loads issued while keys 64-127 are still being exponentiated.
       // P goes to columns 64..127 as bf16 pairs (keys 0-63 -> 64..95,
       // keys 64-127 -> 96..127), i.e. only over scores already read.
-      auto mask_half = [&](uint32_t* v, int half) {
+      auto mask32 = [&](uint32_t* v, int k0) {
         if (!full) {
 #pragma unroll
-          for (int e = 0; e < 64; ++e) {
-            const int key = c0 + half * 64 + e;
+          for (int e = 0; e < 32; ++e) {
+            const int key = c0 + k0 + e;
             if (!(key <= hi_r && key > lo_r && key < p.Lk)) v[e] = __float_as_uint(-INFINITY);
           }
         }
       };
-      auto exp_half = [&](const uint32_t* v, int half, float m_use) {
+      // P of 32 keys -> 16 TMEM columns
+      auto exp32 = [&](const uint32_t* v, uint32_t col, float m_use) {
+        uint32_t pk[16];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float p0 = fast_exp2(fmaf(__uint_as_float(v[c * 32 + e]), p.scale_log2, -m_use));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(v[c * 32 + e + 1]), p.scale_log2, -m_use));
-            l_run += p0 + p1;
-            pk[e >> 1] = pack_bf16(p0, p1);
-          }
-          tc::tmem_st16(tS + 64 + half * 32 + c * 16, pk);
+        for (int e = 0; e < 32; e += 2) {
+          const float p0 = fast_exp2(fmaf(__uint_as_float(v[e]), p.scale_log2, -m_use));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(v[e + 1]), p.scale_log2, -m_use));
+          l_run += p0 + p1;
+          pk[e >> 1] = pack_bf16(p0, p1);
         }
+        tc::tmem_st16(tS + col, pk);
       };
-      float mx = -INFINITY;
+      // the values of a tcgen05.ld are only defined after tcgen05.wait::ld:
+      // an empty asm on each register keeps every use behind the wait
+      auto pin32 = [](uint32_t* v) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) asm volatile("" : "+r"(v[e]));
+      };
+      uint32_t v1[64];
+      float mx;
       {
         uint32_t v[64];
         tc::tmem_ld32(tS, v);
         tc::tmem_ld32(tS + 32, v + 32);
+        tc::tmem_ld32(tS + 64, v1);
+        tc::tmem_ld32(tS + 96, v1 + 32);
         tc::tmem_wait_ld();
-        mask_half(v, 0);
+        pin32(v); pin32(v + 32); pin32(v1); pin32(v1 + 32);
+        mask32(v, 0); mask32(v + 32, 32); mask32(v1, 64); mask32(v1 + 32, 96);
+        float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < 64; ++e) mx = fmaxf(mx, __uint_as_float(v[e]));
+        for (int e = 0; e < 64; e += 2) {
+          m0 = fmaxf(m0, fmaxf(__uint_as_float(v[e]), __uint_as_float(v[e + 1])));
+          m1 = fmaxf(m1, fmaxf(__uint_as_float(v1[e]), __uint_as_float(v1[e + 1])));
+        }
+        mx = fmaxf(m0, m1);
       }
-      uint32_t v1[64];
-      tc::tmem_ld32(tS + 64, v1);
-      tc::tmem_ld32(tS + 96, v1 + 32);
-      tc::tmem_wait_ld();
-      mask_half(v1, 1);
-#pragma unroll
-      for (int e = 0; e < 64; ++e) mx = fmaxf(mx, __uint_as_float(v1[e]));
       const float m_tile = mx * p.scale_log2;
       const bool need = m_tile > m_run + kRescaleLog2;
       if (__any_sync(0xffffffffu, need)) {
@@ -317,19 +326,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_run = m_new;
       }
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      exp_half(v1, 1, m_use);
+      uint32_t v0[64];
+      exp32(v1, 96, m_use);
+      tc::tmem_ld32(tS, v0);  // keys 0-31 again, in flight under the next 32 exponentials
+      exp32(v1 + 32, 112, m_use);
+      tc::tmem_ld32(tS + 32, v0 + 32);
       tc::tmem_wait_st();
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(bar(B_PA + q));
-      {
-        uint32_t v[64];
-        tc::tmem_ld32(tS, v);
-        tc::tmem_ld32(tS + 32, v + 32);
-        tc::tmem_wait_ld();
-        mask_half(v, 0);
-        exp_half(v, 0, m_use);
-      }
+      tc::tmem_wait_ld();
+      pin32(v0); pin32(v0 + 32);
+      mask32(v0, 0); mask32(v0 + 32, 32);
+      exp32(v0, 64, m_use);
+      exp32(v0 + 32, 80, m_use);
       tc::tmem_wait_st();
       tc::tc_fence_before();
       __syncwarp();

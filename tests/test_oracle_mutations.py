@@ -113,6 +113,8 @@ MUTANTS = [
 ]
 
 
+# a planted mistake may overflow on the way to failing its pin (that is the point)
+@pytest.mark.filterwarnings("ignore:overflow encountered:RuntimeWarning")
 @pytest.mark.parametrize("case", MUTANTS, ids=[m[0] for m in MUTANTS])
 def test_pins_catch_mutant(case, golden, monkeypatch):
     _, module, old, new, checks = case

@@ -8,8 +8,10 @@
 // section "隐式序列缩放的技术细节" step 2 (causal attention over the expanded
 // sequence).
 //
-// One CTA = two consecutive 128-row query tiles of one (batch, head, stream
-// group); they share every K/V tile the CTA loads.
+// One CTA = two 128-row query tiles that share every K/V tile the CTA loads:
+// the same rows of two query heads of one GQA group (when the group size is
+// even), so both tiles take exactly the same K/V steps; otherwise two
+// consecutive row tiles of one head. Always of one (batch, stream group).
 //   warps 0-3 / 4-7  softmax warpgroup of query tile 0 / 1, one row per thread
 //               (= TMEM lane): tcgen05.ld of the S row, mask on boundary tiles,
 //               online softmax in base 2, P as bf16 pairs written back into the
@@ -75,6 +77,13 @@ struct TcSmem {
 // p_hi: P of keys 64-127 written; p_lo: P of keys 0-63 written
 enum { B_QF = 0, B_KF = 1, B_VF = 3, B_KE = 5, B_SF = 7, B_PA = 9, B_PB = 11, B_OF = 13 };
 
+// A CTA takes the same query rows of two heads of one GQA group when the group
+// size is even (their K/V steps are identical), else two consecutive row tiles
+// of one head (the second one needs one K/V tile more on the causal diagonal).
+__host__ __device__ __forceinline__ bool fwd_head_pairs(const AttnParams& p) {
+  return (p.Hq / p.Hkv) % 2 == 0;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ,
@@ -94,26 +103,45 @@ __global__ void __launch_bounds__(kThreads, 1)
   // word is cleared: skip the work instead of waiting again.
   if (p.status && *reinterpret_cast<volatile int*>(p.status) == HD_ERR_TIMEOUT) return;
 
-  // ---- problem of this CTA: query tiles 2*pq and 2*pq+1
-  const int bhg = p.B * p.Hq * p.groups;
+  // ---- problem of this CTA: its two query tiles
   const int num_qt = (p.Lq + kBM - 1) / kBM;
-  const int num_pairs = (num_qt + 1) / 2;
-  const int pq = num_pairs - 1 - static_cast<int>(blockIdx.x / bhg);  // heavy pairs first
-  int y = static_cast<int>(blockIdx.x % bhg);
-  const int grp = y % p.groups;
-  y /= p.groups;
-  const int h = y % p.Hq;
-  const int b = y / p.Hq;
-  const int hk = h / (p.Hq / p.Hkv);
+  const bool head_pair = fwd_head_pairs(p);
+  int b, grp, h0, h1, r00, r01;  // batch, stream group; head and first row of tile 0 / 1
+  if (head_pair) {
+    // the same 128 rows of two query heads that share a KV head: both tiles
+    // visit exactly the same K/V tiles
+    const int bhg = p.B * (p.Hq / 2) * p.groups;
+    const int qt = num_qt - 1 - static_cast<int>(blockIdx.x / bhg);  // heavy tiles first
+    int y = static_cast<int>(blockIdx.x % bhg);
+    grp = y % p.groups;
+    y /= p.groups;
+    h0 = 2 * (y % (p.Hq / 2));
+    h1 = h0 + 1;
+    b = y / (p.Hq / 2);
+    r00 = r01 = qt * kBM;
+  } else {
+    // query tiles 2*pq and 2*pq+1 of one head
+    const int bhg = p.B * p.Hq * p.groups;
+    const int num_pairs = (num_qt + 1) / 2;
+    const int pq = num_pairs - 1 - static_cast<int>(blockIdx.x / bhg);  // heavy pairs first
+    int y = static_cast<int>(blockIdx.x % bhg);
+    grp = y % p.groups;
+    y /= p.groups;
+    h0 = h1 = y % p.Hq;
+    b = y / p.Hq;
+    r00 = 2 * pq * kBM;
+    r01 = r00 + kBM;
+  }
+  const int hk = h0 / (p.Hq / p.Hkv);
   const bool intra = p.mode == HD_INTRA;
-  const int jq = (intra && !p.final_only) ? grp * p.Hq + h : h;
+  const int jq0 = (intra && !p.final_only) ? grp * p.Hq + h0 : h0;
+  const int jq1 = (intra && !p.final_only) ? grp * p.Hq + h1 : h1;
   const int jk = intra ? (p.final_only ? p.n - 1 : grp) * p.Hkv + hk : hk;
-  const int r0 = 2 * pq * kBM;
   // K/V tile range [lo_q, hi_q] of each query tile (empty when the tile has no rows)
   int lo[2], hi[2];
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
-    const int rq = r0 + q * kBM;
+    const int rq = q ? r01 : r00;
     if (rq >= p.Lq) {
       lo[q] = 1;
       hi[q] = 0;
@@ -155,7 +183,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int q = 0; q < 2; ++q)
 #pragma unroll
         for (int s = 0; s < NSUB; ++s)
-          tc::tma_load_4d(sQ + q * SM::Q_BYTES + s * kSub, &tmQ, bar(B_QF), s * 64, jq, r0 + q * kBM, b);
+          tc::tma_load_4d(sQ + q * SM::Q_BYTES + s * kSub, &tmQ, bar(B_QF), s * 64, q ? jq1 : jq0,
+                          q ? r01 : r00, b);
       for (int i = 0; i < nkv; ++i) {
         const int st = i & 1;
         if (!tc::mbar_wait(bar(B_KE + st), ((i >> 1) & 1) ^ 1, abort_flag, p.status)) break;
@@ -238,10 +267,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------ softmax warpgroups
     const int q = warp >> 2;  // query tile of this warpgroup
     const int row = tid & 127;
-    const int r = r0 + q * kBM + row;
+    const int rq0 = q ? r01 : r00;  // first row of this warpgroup's tile
+    const int hq = q ? h1 : h0, jq = q ? jq1 : jq0;
+    const int r = rq0 + row;
     const uint32_t tq = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + 256 * q + tq, tO = tS + 128;
-    const int rq0 = r0 + q * kBM;
     const int rq_last = min(rq0 + kBM, p.Lq) - 1;
     const int hi_r = p.a * r + p.bb;
     const int lo_r = hi_r - p.win;
@@ -369,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (r < p.Lq) {
-        const long long li = (static_cast<long long>(b) * p.Hq + h) * p.Sq +
+        const long long li = (static_cast<long long>(b) * p.Hq + hq) * p.Sq +
                              static_cast<long long>(grp) * p.qs_step +
                              static_cast<long long>(r) * p.q_rstride;
         p.lse[li] = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
@@ -454,7 +484,8 @@ cudaError_t launch_tc_d(const AttnParams& p, cudaStream_t stream) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const long long num_qt = (p.Lq + kBM - 1) / kBM;
-  const long long blocks = (num_qt + 1) / 2 * p.B * p.Hq * p.groups;
+  const long long blocks = fwd_head_pairs(p) ? num_qt * p.B * (p.Hq / 2) * p.groups
+                                             : (num_qt + 1) / 2 * p.B * p.Hq * p.groups;
   attn_fwd_tc_kernel<D><<<static_cast<unsigned>(blocks), kThreads, smem, stream>>>(p, mq, mk, mv, mo);
   return cudaGetLastError();
 }

@@ -32,6 +32,7 @@ SMALL = [
     (1, 1, 4, 2, 1, 64, 1),       # one token: S = n
     (2, 130, 2, 6, 3, 64, 64),    # crosses a 128-row tile and a 64-key tile
     (1, 200, 4, 2, 2, 128, 300),  # W > L (window = full causal)
+    (1, 150, 2, 3, 1, 64, 20),    # odd GQA group (3 query heads per KV head)
 ]
 
 

@@ -45,6 +45,7 @@ constexpr int kKN = 128;   // keys per CTA
 constexpr int kQM = 64;    // query rows per iteration
 constexpr int kQS = 3;     // Q / dO stages
 constexpr int kThreads = 480;
+constexpr int kKB = 8;     // key tiles per grid bucket for INTRA problems
 constexpr uint32_t kTmemCols = 512;
 
 template <int D>
@@ -106,11 +107,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (p.status && *reinterpret_cast<volatile int*>(p.status) == HD_ERR_TIMEOUT) return;
 
-  // ---- problem of this CTA: key tile kt of (b, hk, grp); key-tile-major grid,
-  // low key tiles (which see the most queries) first
+  // ---- problem of this CTA: key tile kt of (b, hk, grp). The grid walks
+  // buckets of key tiles, low buckets (which see the most queries) first.
+  // Inside a bucket a problem's key tiles are adjacent, so they run at the
+  // same time and share their Q, dO and dQ tiles in L2. INTRA problems (one
+  // stream each, many of them) take buckets of kKB key tiles; the others one
+  // key tile per bucket (key-tile-major), which measured best for them.
   const int bkg = p.B * p.Hkv * p.groups;
-  const int kt = static_cast<int>(blockIdx.x / bkg);
-  int y = static_cast<int>(blockIdx.x % bkg);
+  const int num_kt = (p.Lk + kKN - 1) / kKN;
+  const int kb = p.groups > 1 ? min(kKB, num_kt) : 1;
+  const int bucket = static_cast<int>(blockIdx.x / (bkg * kb));
+  const int rem = static_cast<int>(blockIdx.x - static_cast<long long>(bucket) * bkg * kb);
+  const int bsize = min(kb, num_kt - bucket * kb);
+  const int kt = bucket * kb + rem % bsize;
+  int y = rem / bsize;
   const int grp = y % p.groups;
   y /= p.groups;
   const int hk = y % p.Hkv;

@@ -18,8 +18,8 @@
 //               upper S columns of TMEM (tcgen05.st). The running max is only raised
 //               when a tile's max exceeds it by more than 2^8, so the O
 //               accumulator is rescaled in TMEM rarely; the final 1/l and LSE
-//               make the result exact either way. The reload of keys 0-63 is
-//               issued while keys 64-127 are still being exponentiated.
+//               make the result exact either way. The row's scores are read
+//               from TMEM once and kept in registers.
 //   warp 8      TMA producer: both Q tiles once, then K and V tiles of 128 keys
 //               into a 2-stage ring (128-byte swizzle). The 4-D tensor maps are
 //               (d, head-or-stream*head, row, batch), so an INTRA stream is read
@@ -285,9 +285,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int c0 = j * kBN;
       const bool full = (c0 + kBN - 1 <= p.a * rq0 + p.bb) &&
                         (c0 > p.a * rq_last + p.bb - p.win) && (c0 + kBN <= p.Lk);
-      // The row's 128 scores are read from TMEM once for the max; keys 64-127
-      // stay in registers for their P, and keys 0-63 are read again, those
-      // loads issued while keys 64-127 are still being exponentiated.
+      // The row's 128 scores are read from TMEM once and stay in registers
+      // (167 registers per thread, under the 168 that 10 warps allow).
       // P goes to columns 64..127 as bf16 pairs (keys 0-63 -> 64..95,
       // keys 64-127 -> 96..127), i.e. only over scores already read.
       auto mask32 = [&](uint32_t* v, int k0) {
@@ -318,9 +317,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 32; ++e) asm volatile("" : "+r"(v[e]));
       };
       uint32_t v1[64];
+      uint32_t v[64];
       float mx;
       {
-        uint32_t v[64];
         tc::tmem_ld32(tS, v);
         tc::tmem_ld32(tS + 32, v + 32);
         tc::tmem_ld32(tS + 64, v1);
@@ -342,34 +341,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float m_new = fmaxf(m_run, m_tile);
         const float alpha = (m_run == -INFINITY) ? 0.f : fast_exp2(m_run - m_new);
         if (t > 0) {
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tc::tmem_ld32(tO + c * 32, o);
+          // 8 columns at a time: all 128 scores of the row are live here
+#pragma unroll 1
+          for (int c = 0; c < D / 8; ++c) {
+            uint32_t o[8];
+            tc::tmem_ld8(tO + c * 8, o);
             tc::tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tc::tmem_st32(tO + c * 32, o);
+            for (int e = 0; e < 8; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tc::tmem_st8(tO + c * 8, o);
           }
         }
         l_run *= alpha;
         m_run = m_new;
       }
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      uint32_t v0[64];
       exp32(v1, 96, m_use);
-      tc::tmem_ld32(tS, v0);  // keys 0-31 again, in flight under the next 32 exponentials
       exp32(v1 + 32, 112, m_use);
-      tc::tmem_ld32(tS + 32, v0 + 32);
       tc::tmem_wait_st();
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(bar(B_PA + q));
-      tc::tmem_wait_ld();
-      pin32(v0); pin32(v0 + 32);
-      mask32(v0, 0); mask32(v0 + 32, 32);
-      exp32(v0, 64, m_use);
-      exp32(v0 + 32, 80, m_use);
+      exp32(v, 64, m_use);
+      exp32(v + 32, 80, m_use);
       tc::tmem_wait_st();
       tc::tc_fence_before();
       __syncwarp();

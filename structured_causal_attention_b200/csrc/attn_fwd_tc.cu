@@ -32,7 +32,7 @@
 //               S = Q K^T (M=128, N=128, both operands from shared memory);
 //               O += P V (M=128, N=D, P from TMEM, V MN-major from its TMA tile),
 //               issued in two halves of 64 keys: the softmax signals P of keys
-//               64-127 before it reloads and exponentiates keys 0-63, so half
+//               64-127 before it exponentiates keys 0-63, so half
 //               of PV runs under the rest of the softmax.
 // MMAs from one thread execute in order, so when S_q(j) is complete, PV_q(j-1)
 // (issued before it) has finished reading P and updating O: the softmax may

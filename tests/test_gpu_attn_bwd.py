@@ -32,6 +32,7 @@ SMALL = [
     (1, 1, 4, 2, 1, 64, 1),
     (1, 130, 2, 6, 3, 64, 64),
     (1, 100, 4, 2, 2, 128, 300),
+    (1, 1200, 2, 2, 1, 64, 100),  # 10 key tiles per INTRA stream: a partial grid bucket
 ]
 
 

@@ -45,7 +45,7 @@ constexpr int kKN = 128;   // keys per CTA
 constexpr int kQM = 64;    // query rows per iteration
 constexpr int kQS = 3;     // Q / dO stages
 constexpr int kThreads = 480;
-constexpr int kKB = 8;     // key tiles per grid bucket for INTRA problems
+constexpr int kKB = 8;     // key tiles per grid bucket (INTRA, short windows)
 constexpr uint32_t kTmemCols = 512;
 
 template <int D>
@@ -110,12 +110,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- problem of this CTA: key tile kt of (b, hk, grp). The grid walks
   // buckets of key tiles, low buckets (which see the most queries) first.
   // Inside a bucket a problem's key tiles are adjacent, so they run at the
-  // same time and share their Q, dO and dQ tiles in L2. INTRA problems (one
-  // stream each, many of them) take buckets of kKB key tiles; the others one
-  // key tile per bucket (key-tile-major), which measured best for them.
+  // same time and share their Q, dO and dQ tiles in L2. Buckets of kKB key
+  // tiles for INTRA problems (one stream each, many of them) and for windows
+  // short against the sequence (key tiles of nearly equal work); otherwise
+  // one key tile per bucket (key-tile-major), which measured best there.
   const int bkg = p.B * p.Hkv * p.groups;
   const int num_kt = (p.Lk + kKN - 1) / kKN;
-  const int kb = p.groups > 1 ? min(kKB, num_kt) : 1;
+  const bool bucketed = p.groups > 1 || 4LL * p.win <= p.Lk;
+  const int kb = bucketed ? min(kKB, num_kt) : 1;
   const int bucket = static_cast<int>(blockIdx.x / (bkg * kb));
   const int rem = static_cast<int>(blockIdx.x - static_cast<long long>(bucket) * bkg * kb);
   const int bsize = min(kb, num_kt - bucket * kb);

@@ -272,6 +272,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = tid & 127;
     const int c = c0 + row;
     const uint32_t tq = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    // The query rows this thread's key is visible to, r_lo .. r_hi (empty when
+    // r_lo > r_hi), from the visibility rule c <= a*r + bb, c > a*r + bb - win,
+    // r < Lq, c < Lk; fixed for the whole CTA. c - bb + win - 1 >= 0 always,
+    // since win >= a (a window spans at least one token's n positions).
+    int r_lo = 1, r_hi = 0;
+    if (c < p.Lk) {
+      r_lo = (c - p.bb <= 0) ? 0 : (c - p.bb + p.a - 1) / p.a;
+      const long long num = static_cast<long long>(c) - p.bb + p.win - 1;
+      r_hi = static_cast<int>(min(static_cast<long long>(p.Lq - 1), num / p.a));
+    }
     bool ok = true;
     for (int it = 0; it < total; ++it) {
       const int x = it & 1, st = it % kQS;
@@ -290,12 +300,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // The mask is a separate pass (score -> -inf, so P and dS become 0):
         // a test inside the arithmetic loop below would serialise it.
         if (!full) {
+          const int elo = r_lo - (rq0 + sw * 32), ehi = r_hi - (rq0 + sw * 32);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int r = rq0 + sw * 32 + e;
-            const int hi = p.a * r + p.bb;
-            if (!(r < p.Lq && c <= hi && c > hi - p.win && c < p.Lk)) sr[e] = __float_as_uint(-INFINITY);
-          }
+          for (int e = 0; e < 32; ++e)
+            if (e < elo || e > ehi) sr[e] = __float_as_uint(-INFINITY);
         }
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {

@@ -13,7 +13,7 @@
 //   dV  += P^T dO     (M 128 keys, N D)            } accumulated in TMEM across
 //   dK  += dS^T Q     (M 128 keys, N D)            } the whole group
 //   dQ^T = K^T dS^T   (M D, N 64 queries)           into the S^T buffer
-// Roles (14 warps):
+// Roles (15 warps):
 //   warps 0-7   two warpgroups, one key row per thread, each taking 32 of the
 //               64 query columns: P^T = exp2(S^T - LSE), dS^T = P^T (dP^T - D),
 //               written as bf16 into shared memory in the MMA operand layout;
@@ -30,6 +30,8 @@
 // one elected lane issues. The two groups wait on different barriers (P^T
 // written vs. the next stage loaded and its buffer free), so each has its own
 // warp; their hand-offs go through the barriers below, not issue order.
+// The grid walks key tiles heavy-first, in buckets that keep a problem's
+// neighbouring key tiles running together where that helps L2 reuse (below).
 // Every mbarrier wait is bounded (HD_ERR_TIMEOUT, then every role leaves).
 #include <cuda.h>
 

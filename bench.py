@@ -471,9 +471,9 @@ DESCRIPTIONS = {
 # the same build (dram__bytes_read.sum + dram__bytes_write.sum); None when the
 # kernel changed after that capture.
 NCU_TRAFFIC = {
-    ("step", "bwd_cross_full"): 4.810e9,  # attn_bwd_tc_kernel, profiles/attn_bwd_tc_kernel_cross_full_intra_train.md
-    ("lm_head", "lm_head_ce"): 2.280e9,   # lm_head_ce_kernel, profiles/lm_head_ce_kernel_lm_head.md
-    ("rope", "rope"): 2.628e9,            # rope_kernel, profiles/rope_kernel_rope.md
+    ("step", "bwd_cross_full"): 4.810e9,  # attn_bwd_tc_kernel
+    ("lm_head", "lm_head_ce"): 2.280e9,   # lm_head_ce_kernel
+    ("rope", "rope"): 2.628e9,            # rope_kernel
 }
 
 

@@ -293,9 +293,10 @@ int hd_decode_attn_final(const void* q, const void* k_cache, const void* v_cache
  * allocates nothing and calls no allocating routine.
  *   - Sizes whose hd_decode_workspace_bytes(...) exceeds
  *     HD_DECODE_NOALLOC_SCRATCH_BYTES are rejected with HD_ERR_UNSUPPORTED.
- *   - The first call on each device looks up the array's device address
- *     (with that device current) and caches it; make that first call before
- *     any stream capture.
+ *   - Every call looks up the array's device address on the calling device
+ *     (cudaGetSymbolAddress, which allocates nothing) before it launches. The
+ *     first call on a device may also load the library's device code there:
+ *     make that first call before any stream capture.
  *   - All calls on a device share the array, which keeps the last call's
  *     contents; nothing in it needs to start at zero. Calls that overlap on
  *     the GPU (two streams, or unordered host threads) race on it: order them.

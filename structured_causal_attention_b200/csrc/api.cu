@@ -4,7 +4,6 @@
 #include <math.h>
 
 #include <cmath>
-#include <mutex>
 
 #include "hd_common.cuh"
 #include "launch.h"
@@ -16,22 +15,14 @@ __device__ int g_status_word;
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-int* g_status_ptr[kMaxDevices] = {};
-std::mutex g_status_mu;
-
-// Device address of the status word on the current device (looked up once per
-// device; host code must not pass the symbol itself to a kernel).
+// Device address of the status word on the current device. Host code must not
+// pass the symbol itself to a kernel: it names a host-side stand-in. The
+// address is looked up on every call (a map lookup in the runtime), so it is
+// never stale, not even after the device was reset.
 int* status_ptr() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_status_mu);
-  if (!g_status_ptr[dev]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_status_word) != cudaSuccess) return nullptr;
-    g_status_ptr[dev] = static_cast<int*>(ptr);
-  }
-  return g_status_ptr[dev];
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_status_word) != cudaSuccess) return nullptr;
+  return static_cast<int*>(ptr);
 }
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
@@ -117,11 +108,23 @@ size_t packed_rows(int B, int L, int n, int Hq, int final_only) {
 
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? HD_OK : HD_ERR_CUDA; }
 
+// Streaming multiprocessors of the current device; 148 (a B200) when no device
+// can be queried, so that workspace sizes can still be computed without one.
+int sm_count() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) {
+    cudaGetLastError();  // clear the error the failed query recorded
+    return 148;
+  }
+  return sms;
+}
+
 // Split-K partials for `rows` query rows per (sequence, KV head) against up to
 // `keys` keys: unnormalised O (fp32 [.., D]) and (max, sum) pairs.
 size_t decode_partials_bytes(int B, int rows, long long keys, int Hkv, int D) {
   int mt = 0, splits = 0, chunk = 0;
-  decode_split_plan(B, rows, keys, Hkv, &mt, &splits, &chunk);
+  decode_split_plan(B, rows, keys, Hkv, sm_count(), &mt, &splits, &chunk);
   const size_t prow = static_cast<size_t>(B) * Hkv * mt * 16 * splits;
   return align256(prow * static_cast<size_t>(D) * 4) + align256(prow * 2 * 4);
 }
@@ -189,8 +192,8 @@ int decode_call(const void* q, const void* k_cache, const void* v_cache, const i
     p.mode = HD_CROSS_FULL;
   }
   p.rows = p.nq * (Hq / Hkv);
-  decode_split_plan(B, p.rows, static_cast<long long>(Tcap) * p.kpt, Hkv, &p.mt, &p.splits,
-                    &p.chunk);
+  decode_split_plan(B, p.rows, static_cast<long long>(Tcap) * p.kpt, Hkv, sm_count(), &p.mt,
+                    &p.splits, &p.chunk);
   const size_t prow = static_cast<size_t>(B) * Hkv * p.mt * 16 * p.splits;
   p.part_o = static_cast<float*>(workspace);
   p.part_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(prow * D * 4));

@@ -327,10 +327,11 @@ cudaError_t launch_decode_d(const DecodeParams& p, cudaStream_t stream) {
 
 }  // namespace
 
-void decode_split_plan(int B, int rows, long long keys, int Hkv, int* mt, int* splits, int* chunk) {
+void decode_split_plan(int B, int rows, long long keys, int Hkv, int sms, int* mt, int* splits,
+                       int* chunk) {
   const int m = (rows + 15) / 16;
   const long long units = static_cast<long long>(B) * Hkv * m;
-  const long long target = 148LL * 2 * 4;  // 4 waves of 2 resident CTAs per SM
+  const long long target = static_cast<long long>(sms) * 2 * 4;  // 4 waves of 2 resident CTAs per SM
   long long sp = (target + units - 1) / units;
   // at least 8 blocks (512 keys) per split, so that short caches are not cut
   // into many tiny chunks that the combine step then has to walk

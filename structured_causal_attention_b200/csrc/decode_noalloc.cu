@@ -16,8 +16,6 @@
 // one device (two streams, or two host threads without ordering) race on the
 // array and corrupt each other's results: order such calls on one stream or
 // with events.
-#include <mutex>
-
 #include "hd_common.cuh"
 #include "launch.h"
 
@@ -26,24 +24,15 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_decode_scratch[HD_DECODE_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDev = 64;
-void* g_scratch_addr[kMaxDev] = {};
-std::mutex g_scratch_mu;
-
 // Device address of the scratch on the current device. In host code the
-// symbol names a host-side shadow, not device memory, so the address is
-// looked up once per device (with that device current) and cached.
+// symbol names a host-side stand-in, not device memory, so the address is
+// looked up with the calling device current. The lookup is repeated on every
+// call (a map lookup in the runtime), so it never goes stale, not even after
+// a device reset.
 int scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return HD_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDev) return HD_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess || !ptr) return HD_ERR_CUDA;
-    g_scratch_addr[dev] = ptr;
-  }
-  *out = g_scratch_addr[dev];
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess || !ptr) return HD_ERR_CUDA;
+  *out = ptr;
   return HD_OK;
 }
 

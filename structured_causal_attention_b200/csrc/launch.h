@@ -37,8 +37,10 @@ struct DecodeParams {
 };
 
 // Number of splits / chunk length the decode launcher uses for `rows` query
-// rows per (sequence, KV head) against up to `keys` keys.
-void decode_split_plan(int B, int rows, long long keys, int Hkv, int* mt, int* splits, int* chunk);
+// rows per (sequence, KV head) against up to `keys` keys on a GPU of `sms`
+// streaming multiprocessors.
+void decode_split_plan(int B, int rows, long long keys, int Hkv, int sms, int* mt, int* splits,
+                       int* chunk);
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
 
 struct RopeParams {

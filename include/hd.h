@@ -58,7 +58,9 @@ typedef enum {
   HD_ERR_UNSUPPORTED = 2, /* valid arguments this build does not cover (e.g. D not in {64,128}) */
   HD_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
   HD_ERR_TIMEOUT = 4,     /* device status: a bounded wait inside a kernel gave up */
-  HD_ERR_DEVICE_INDEX = 5 /* device status: a token id outside [0, V) (row left zero) */
+  HD_ERR_DEVICE_INDEX = 5 /* device status: an index read on the device was out of range (a token
+                             id, seqlen, label or offset; in the checked build also a computed
+                             load/store index) */
 } hd_status;
 
 typedef enum { HD_INTRA = 0, HD_CROSS_FULL = 1, HD_CROSS_WINDOW = 2 } hd_mode;
@@ -68,8 +70,18 @@ const char* hd_status_string(int status);
 
 /* Library ABI version: (major << 16) | minor. Minor 1 added RoPE, the
  * final-stream readout, the LM-head cross-entropy and its gradients,
- * final-stream-only decode and the bounded-wait self-test. */
+ * final-stream-only decode and the bounded-wait self-test; minor 2 added
+ * hd_build_flags. */
 int hd_version(void);
+
+/* How this copy of the library was built (no counterpart on the pages), a bit
+ * mask: HD_BUILD_CHECK_BOUNDS is set in the checked build (libhd_checked.so,
+ * compiled with HD_CHECK_BOUNDS), whose kernels test every computed index of a
+ * plain (non-TMA) load or store against the size of its buffer. An index out
+ * of range records HD_ERR_DEVICE_INDEX in the device status word and its access
+ * is skipped; nothing traps. The normal build (libhd.so) has no such checks. */
+#define HD_BUILD_CHECK_BOUNDS 1
+int hd_build_flags(void);
 
 /*
  * hd_expand_embed - interleaved n-table embedding gather.

@@ -12,6 +12,8 @@ import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libhd.so")
+# the same library built with HD_CHECK_BOUNDS (bounds-checked kernels), for tests
+LIB_CHECKED_PATH = os.path.join(HERE, "libhd_checked.so")
 
 HD_OK = 0
 HD_ERR_INVALID_ARG = 1
@@ -29,6 +31,7 @@ _D = ctypes.c_double
 SIGNATURES = {
     "hd_status_string": (ctypes.c_char_p, [_I]),
     "hd_version": (_I, []),
+    "hd_build_flags": (_I, []),
     "hd_expand_embed": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
     "hd_rope_expanded": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _D, _P]),
     "hd_final_readout": (_I, [_P, _P, _I, _I, _I, _I, _I, _P]),
@@ -53,6 +56,7 @@ SIGNATURES = {
 }
 
 _lib = None
+_lib_checked = None
 
 
 class HDError(RuntimeError):
@@ -61,20 +65,32 @@ class HDError(RuntimeError):
         super().__init__(f"{what}: {status_string(status)}")
 
 
+def _load(path):
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with `python -m structured_causal_attention_b200.build`")
+    handle = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(handle, name)
+        fn.restype = res
+        fn.argtypes = args
+    return handle
+
+
 def lib():
     """Load libhd.so once; raise if it is absent (no fallback exists)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(
-                f"{LIB_PATH} is missing: build it with `python -m structured_causal_attention_b200.build`")
-        handle = ctypes.CDLL(LIB_PATH)
-        for name, (res, args) in SIGNATURES.items():
-            fn = getattr(handle, name)
-            fn.restype = res
-            fn.argtypes = args
-        _lib = handle
+        _lib = _load(LIB_PATH)
     return _lib
+
+
+def lib_checked():
+    """Load the checked build, libhd_checked.so (same ABI, bounds-checked kernels)."""
+    global _lib_checked
+    if _lib_checked is None:
+        _lib_checked = _load(LIB_CHECKED_PATH)
+    return _lib_checked
 
 
 def status_string(status: int) -> str:

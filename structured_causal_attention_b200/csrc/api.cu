@@ -63,6 +63,9 @@ AttnParams make_params(const void* q, const void* k, const void* v, int B, int L
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634074f;
   p.status = status_ptr();
+  p.ext_q = static_cast<long long>(B) * p.Sq * Hq * D;
+  p.ext_lse = static_cast<long long>(B) * Hq * p.Sq;
+  p.ext_kv = static_cast<long long>(B) * p.S * Hkv * D;
   if (mode == HD_INTRA) {
     // each stream is its own causal problem over the L tokens
     p.groups = final_only ? 1 : n;
@@ -195,6 +198,10 @@ int decode_call(const void* q, const void* k_cache, const void* v_cache, const i
   decode_split_plan(B, p.rows, static_cast<long long>(Tcap) * p.kpt, Hkv, sm_count(), &p.mt,
                     &p.splits, &p.chunk);
   const size_t prow = static_cast<size_t>(B) * Hkv * p.mt * 16 * p.splits;
+  p.ext_q = static_cast<long long>(B) * p.nq * Hq * D;
+  p.ext_lse = static_cast<long long>(B) * Hq * p.nq;
+  p.ext_cache = static_cast<long long>(B) * Tcap * n * Hkv * D;
+  p.ext_part = static_cast<long long>(prow);
   p.part_o = static_cast<float*>(workspace);
   p.part_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(prow * D * 4));
   p.scale_log2 = scale * 1.4426950408889634074f;
@@ -220,7 +227,15 @@ const char* hd_status_string(int status) {
   }
 }
 
-int hd_version(void) { return (1 << 16) | 1; }
+int hd_version(void) { return (1 << 16) | 2; }
+
+int hd_build_flags(void) {
+#ifdef HD_CHECK_BOUNDS
+  return HD_BUILD_CHECK_BOUNDS;
+#else
+  return 0;
+#endif
+}
 
 int hd_expand_embed(const int32_t* ids, const void* tables, void* out, int B, int L, int n, int V,
                     int d, int elem_bytes, void* stream) {
@@ -273,7 +288,7 @@ int hd_final_readout(const void* x, void* out, int B, int L, int n, int d, int e
   const long long row_bytes = static_cast<long long>(d) * elem_bytes;
   if (row_bytes % 16 != 0) return HD_ERR_UNSUPPORTED;
   return from_cuda(launch_final_readout(x, out, static_cast<long long>(B) * L, n, row_bytes,
-                                        static_cast<cudaStream_t>(stream)));
+                                        status_ptr(), static_cast<cudaStream_t>(stream)));
 }
 
 size_t hd_lm_head_ce_workspace_bytes(int B, int L, int V) {
@@ -390,6 +405,7 @@ int hd_attn_bwd(const void* q, const void* k, const void* v, const void* out, co
   p.lse2p = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(rows * D * 4));
   p.deltap = reinterpret_cast<float*>(reinterpret_cast<char*>(p.lse2p) + align256(npk * 4));
   p.lq_pad = static_cast<int>(pad64(p.Lq));
+  p.ext_packed = static_cast<long long>(npk);
   return from_cuda(launch_attn_bwd(p, static_cast<cudaStream_t>(stream)));
 }
 

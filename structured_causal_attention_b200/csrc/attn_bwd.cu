@@ -33,7 +33,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const AttnParams p) {
   const int sub = lane / LPR, sl = lane % LPR;
   const long long row = (static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + warp) * RPW + sub;
   const long long total = static_cast<long long>(p.B) * p.Sq * p.Hq;
-  const bool valid = row < total;
+  const bool valid = row < total && in_bounds(row * D + 8 * sl, 8, p.ext_q, p.status);
   float acc = 0.f;
   if (valid) {
     const uint4 ov = __ldcs(reinterpret_cast<const uint4*>(p.o + row * D) + sl);
@@ -59,12 +59,14 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const AttnParams p) {
   const long long grp = intra_groups ? i % p.n : 0;
   const long long r = intra_groups ? i / p.n : i;
   const long long pk = ((b * p.Hq + h) * p.groups + grp) * p.lq_pad;
-  if (sl == 0) {
+  if (sl == 0 && in_bounds(pk + r, 1, p.ext_packed, p.status) &&
+      in_bounds((b * p.Hq + h) * p.Sq + i, 1, p.ext_lse, p.status)) {
     p.deltap[pk + r] = acc;
     p.lse2p[pk + r] = p.lse[(b * p.Hq + h) * p.Sq + i] * 1.4426950408889634074f;
   }
   if (r == p.Lq - 1) {  // zero the padding rows after the problem's last row
     for (int j = sl; j < p.lq_pad - p.Lq; j += LPR) {
+      if (!in_bounds(pk + p.Lq + j, 1, p.ext_packed, p.status)) break;
       p.deltap[pk + p.Lq + j] = 0.f;
       p.lse2p[pk + p.Lq + j] = 0.f;
     }
@@ -83,6 +85,7 @@ __global__ void bwd_zero_unread_kv_kernel(const AttnParams p) {
   if (row >= total) return;
   const long long pos = (row / p.Hkv) % p.S;
   if (pos % p.n == p.n - 1) return;
+  if (!in_bounds(row * p.D, p.D, p.ext_kv, p.status)) return;
   uint2* zk = reinterpret_cast<uint2*>(p.dk + row * p.D);
   uint2* zv = reinterpret_cast<uint2*>(p.dv + row * p.D);
   for (int c = lane; c < p.D / 4; c += 32) {
@@ -93,7 +96,7 @@ __global__ void bwd_zero_unread_kv_kernel(const AttnParams p) {
 
 __global__ void bwd_dq_kernel(const AttnParams p, long long n8) {
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= n8) return;
+  if (i >= n8 || !in_bounds(8 * i, 8, p.ext_q, p.status)) return;
   const float4 a = reinterpret_cast<const float4*>(p.dq_acc)[2 * i];
   const float4 c = reinterpret_cast<const float4*>(p.dq_acc)[2 * i + 1];
   uint4 out;

@@ -187,6 +187,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int h = iter_head(it), rq0 = iter_row0(it), jq = jq_of(h);
       if (lane == 0) {
         const long long pk = ((static_cast<long long>(b) * p.Hq + h) * p.groups + grp) * p.lq_pad + rq0;
+        if (!in_bounds(pk, kQM, p.ext_packed, p.status)) {  // checked build only
+          *abort_flag = 1;
+          break;
+        }
         tc::mbar_expect_tx(bar(B_QF + st), 2 * NSUB * SM::QSUB + 2 * kQM * 4);
 #pragma unroll
         for (int s = 0; s < NSUB; ++s) {

@@ -396,7 +396,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const long long li = (static_cast<long long>(b) * p.Hq + hq) * p.Sq +
                              static_cast<long long>(grp) * p.qs_step +
                              static_cast<long long>(r) * p.q_rstride;
-        p.lse[li] = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
+        if (in_bounds(li, 1, p.ext_lse, p.status))
+          p.lse[li] = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
       }
       tc::fence_async_smem();
     }

@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
   const long long part_row0 = (static_cast<long long>(b) * p.Hkv + hk) * rows_pad + mt * 16;
 
   if (cs >= ce) {  // nothing to read in this chunk
-    if (tid < 16) {
+    if (tid < 16 && in_bounds((part_row0 + tid) * p.splits + split, 1, p.ext_part, p.status)) {
       float* ml = p.part_ml + ((part_row0 + tid) * p.splits + split) * 2;
       ml[0] = -INFINITY;
       ml[1] = 0.f;
@@ -87,8 +87,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
     const int lr = i / RC, ch = i % RC, row = mt * 16 + lr;
     const bool valid = row < p.rows;
     const int s = valid ? row / g : 0, j = valid ? row % g : 0;
-    const __nv_bfloat16* src = p.q + ((static_cast<long long>(b) * p.nq + s) * p.Hq + hk * g + j) * D + ch * 8;
-    cp_async16(sQ + swz(lr, ch, RC), src, valid ? 16 : 0);
+    const long long qi = ((static_cast<long long>(b) * p.nq + s) * p.Hq + hk * g + j) * D + ch * 8;
+    const bool inb = in_bounds(qi, 8, p.ext_q, p.status);
+    cp_async16(sQ + swz(lr, ch, RC), p.q + (inb ? qi : 0), (valid && inb) ? 16 : 0);
   }
   const long long kv_rs = static_cast<long long>(p.Hkv) * D;
   const __nv_bfloat16* kg = p.kc + (static_cast<long long>(b) * p.Tcap * p.n * p.Hkv + hk) * D;
@@ -101,9 +102,10 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
       const int row = i / RC, ch = i % RC, c = base + row;
       const long long pos = p.kres + static_cast<long long>(min(c, ce - 1)) * p.kstride;
       const long long off = pos * kv_rs + ch * 8;
-      const int nb = c < ce ? 16 : 0;
-      cp_async16(dk + swz(row, ch, RC), kg + off, nb);
-      cp_async16(dv + swz(row, ch, RC), vg + off, nb);
+      const bool inb = in_bounds((kg - p.kc) + off, 8, p.ext_cache, p.status);
+      const int nb = (c < ce && inb) ? 16 : 0;
+      cp_async16(dk + swz(row, ch, RC), inb ? kg + off : p.kc, nb);
+      cp_async16(dv + swz(row, ch, RC), inb ? vg + off : p.vc, nb);
     }
   };
   load_blk(0, 0);
@@ -258,6 +260,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
       lt += f * mbuf[(w * 16 + lr) * RS + D + 1];
     }
     const long long prow_i = (part_row0 + lr) * p.splits + split;
+    if (!in_bounds(prow_i, 1, p.ext_part, p.status)) continue;
     p.part_o[prow_i * D + col] = acc;
     if (col == 0) {
       p.part_ml[prow_i * 2] = mx;
@@ -278,6 +281,11 @@ __global__ void decode_combine_kernel(const DecodeParams p) {
   const int g = p.Hq / p.Hkv;
   const int s = row / g, h = hk * g + row % g;  // s local to the nq query streams
   const long long prow = (static_cast<long long>(b) * p.Hkv + hk) * (p.mt * 16) + row;
+  const long long oi = ((static_cast<long long>(b) * p.nq + s) * p.Hq + h) * D;
+  const long long li = (static_cast<long long>(b) * p.Hq + h) * p.nq + s;
+  if (!in_bounds(prow * p.splits, p.splits, p.ext_part, p.status) || !in_bounds(oi, D, p.ext_q, p.status) ||
+      !in_bounds(li, 1, p.ext_lse, p.status))
+    return;
   const bool ok = seq_ok(p.seqlen[b], p.Tcap);
 
   float mx = -INFINITY;
@@ -302,12 +310,10 @@ __global__ void decode_combine_kernel(const DecodeParams p) {
     for (int i = 0; i < PER; ++i) acc[i] += f * po[lane + 32 * i];
   }
   const float inv = (ok && lt > 0.f) ? 1.f / lt : 0.f;
-  __nv_bfloat16* out = p.o + ((static_cast<long long>(b) * p.nq + s) * p.Hq + h) * D;
+  __nv_bfloat16* out = p.o + oi;
 #pragma unroll
   for (int i = 0; i < PER; ++i) out[lane + 32 * i] = __float2bfloat16_rn(acc[i] * inv);
-  if (lane == 0)
-    p.lse[(static_cast<long long>(b) * p.Hq + h) * p.nq + s] =
-        (ok && lt > 0.f) ? (mx + __log2f(lt)) * kLn2 : -INFINITY;
+  if (lane == 0) p.lse[li] = (ok && lt > 0.f) ? (mx + __log2f(lt)) * kLn2 : -INFINITY;
 }
 
 template <int D>

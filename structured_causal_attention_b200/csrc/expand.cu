@@ -39,6 +39,10 @@ __global__ void __launch_bounds__(256) expand_kernel(const int32_t* __restrict__
       for (long long i = lane; i < nvec; i += 32) dst[i] = z;
       continue;
     }
+    if (!in_bounds((static_cast<long long>(s) * V + id) * row_bytes, row_bytes,
+                   static_cast<long long>(n) * V * row_bytes, status) ||
+        !in_bounds(row * row_bytes, row_bytes, nrows * row_bytes, status))
+      continue;
     const Vec* src = reinterpret_cast<const Vec*>(
         tables + (static_cast<long long>(s) * V + id) * row_bytes);
     long long i = lane;

@@ -20,6 +20,22 @@ __device__ __forceinline__ void record_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Bounds check of a computed index, compiled in only in the checked build
+// (HD_CHECK_BOUNDS): an access of elements [i, i + n) of a buffer of `ext`
+// elements that does not fit records HD_ERR_DEVICE_INDEX and returns false, and
+// the caller skips the access. In the normal build it is constant true and
+// costs nothing.
+__device__ __forceinline__ bool in_bounds(long long i, long long n, long long ext, int* status) {
+#ifdef HD_CHECK_BOUNDS
+  if (i >= 0 && n >= 0 && i + n <= ext) return true;
+  record_status(status, HD_ERR_DEVICE_INDEX);
+  return false;
+#else
+  (void)i; (void)n; (void)ext; (void)status;
+  return true;
+#endif
+}
+
 // ------------------------------------------------------------- attention problem
 // One attention "problem" is a (batch, query head, stream-group) triple whose
 // query rows r = 0..Lq-1 and key rows c = 0..Lk-1 are addressed with constant
@@ -60,6 +76,11 @@ struct AttnParams {
   int k_rstride;
   float scale;
   float scale_log2;     // scale * log2(e)
+  // allocated elements, for the checked build's bounds checks
+  long long ext_q;      // q, out, dout, dq, dq_acc: B * Sq * Hq * D
+  long long ext_lse;    // lse: B * Hq * Sq
+  long long ext_kv;     // k, v, dk, dv: B * S * Hkv * D
+  long long ext_packed; // lse2p, deltap: packed rows
 };
 
 __device__ __forceinline__ bool key_visible(const AttnParams& p, int r, int c) {

@@ -34,6 +34,11 @@ struct DecodeParams {
   int kstride, kres, kpt;
   int rows, mt, splits, chunk;             // rows = nq*(Hq/Hkv); chunk keys per split
   float scale_log2;
+  // allocated elements, for the checked build's bounds checks
+  long long ext_q;      // q, o: B * nq * Hq * D
+  long long ext_lse;    // lse: B * Hq * nq
+  long long ext_cache;  // each cache: B * Tcap * n * Hkv * D
+  long long ext_part;   // partial rows: B * Hkv * mt * 16 * splits
 };
 
 // Number of splits / chunk length the decode launcher uses for `rows` query
@@ -76,7 +81,7 @@ cudaError_t launch_lm_head_ce_bwd(LmHeadParams p, const void* x, const void* w, 
 cudaError_t launch_lm_head_ce(LmHeadParams p, const void* x, const void* w, int n, int num_sms,
                               cudaStream_t stream);
 cudaError_t launch_final_readout(const void* x, void* out, long long rows, int n,
-                                 long long row_bytes, cudaStream_t stream);
+                                 long long row_bytes, int* status, cudaStream_t stream);
 
 cudaError_t launch_wait_timeout(long long limit_cycles, int* status, cudaStream_t stream);
 

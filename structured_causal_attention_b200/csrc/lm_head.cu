@@ -209,7 +209,8 @@ __global__ void __launch_bounds__(kLThreads, 1)
               g1 = (live && v + 1 < p.V) ? g1 : 0.f;
               pk[j >> 1] = pack_bf16(g0, g1);
             }
-            if (row[h] < p.R) {
+            if (row[h] < p.R &&
+                in_bounds(static_cast<long long>(row[h]) * p.g_ld + v0 + c * 32, 32, p.R * p.g_ld, p.status)) {
               uint4* dst = reinterpret_cast<uint4*>(grow + c * 32);
 #pragma unroll
               for (int q4 = 0; q4 < 4; ++q4)
@@ -243,7 +244,8 @@ __global__ void __launch_bounds__(kLThreads, 1)
             l = l * fast_exp2(m - mn) + s;
             m = mn;
           }
-          if (row[h] < p.R) {
+          if (row[h] < p.R && in_bounds(static_cast<long long>(p.nvt + w.vt) * p.R + row[h], 1,
+                                        2LL * p.nvt * p.R, p.status)) {
             p.part[static_cast<long long>(w.vt) * p.R + row[h]] = m;
             p.part[static_cast<long long>(p.nvt + w.vt) * p.R + row[h]] = l;
             if (lo >= 0 && lo < kLV) p.pick[row[h]] = picked;
@@ -395,15 +397,16 @@ __global__ void __launch_bounds__(kGThreads, 1)
         tc::tmem_ld32(tq + kGN * buf + c * 32, x);
         tc::tmem_wait_ld();
         const int col = n0 + c * 32;
-        if (r < p.M && col < p.N) {
+        const long long ci = static_cast<long long>(r) * p.ldc + col;
+        if (r < p.M && col < p.N && in_bounds(ci, 32, static_cast<long long>(p.M) * p.ldc, p.status)) {
           if (p.c_fp32) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.c) + r * p.ldc + col);
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.c) + ci);
 #pragma unroll
             for (int q4 = 0; q4 < 8; ++q4)
               dst[q4] = make_float4(__uint_as_float(x[4 * q4]) * p.scale, __uint_as_float(x[4 * q4 + 1]) * p.scale,
                                     __uint_as_float(x[4 * q4 + 2]) * p.scale, __uint_as_float(x[4 * q4 + 3]) * p.scale);
           } else {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.c) + r * p.ldc + col);
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.c) + ci);
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
               const float* f = reinterpret_cast<const float*>(x + 8 * q4);
@@ -451,12 +454,15 @@ __global__ void lm_head_combine_kernel(const LmHeadParams p) {
 // out[b, t, :] = x[b, t*n + n-1, :]: one warp per output row, 16-byte vectors.
 __global__ void __launch_bounds__(256) final_readout_kernel(const uint8_t* __restrict__ x,
                                                             uint8_t* __restrict__ out, long long rows,
-                                                            int n, long long row_bytes) {
+                                                            int n, long long row_bytes, int* status) {
   const int lane = threadIdx.x & 31;
   const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
   const long long nvec = row_bytes / 16;
   for (long long r = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
        r < rows; r += warps) {
+    if (!in_bounds((r * n + n - 1) * row_bytes, row_bytes, rows * n * row_bytes, status) ||
+        !in_bounds(r * row_bytes, row_bytes, rows * row_bytes, status))
+      continue;
     const uint4* src = reinterpret_cast<const uint4*>(x + (r * n + n - 1) * row_bytes);
     uint4* dst = reinterpret_cast<uint4*>(out + r * row_bytes);
     long long i = lane;
@@ -609,11 +615,11 @@ cudaError_t launch_lm_head_ce_bwd(LmHeadParams p, const void* x, const void* w, 
 }
 
 cudaError_t launch_final_readout(const void* x, void* out, long long rows, int n,
-                                 long long row_bytes, cudaStream_t stream) {
+                                 long long row_bytes, int* status, cudaStream_t stream) {
   long long blocks = (rows + 7) / 8;
   if (blocks > 148LL * 16) blocks = 148LL * 16;
   final_readout_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-      static_cast<const uint8_t*>(x), static_cast<uint8_t*>(out), rows, n, row_bytes);
+      static_cast<const uint8_t*>(x), static_cast<uint8_t*>(out), rows, n, row_bytes, status);
   return cudaGetLastError();
 }
 

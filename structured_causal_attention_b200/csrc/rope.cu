@@ -108,6 +108,8 @@ __global__ void __launch_bounds__(kRopeThreads) rope_kernel(RopeParams p) {
       __sincosf(static_cast<float>(red), &s[e], &c[e]);  // abs error < 4e-7 on [-pi, pi]
     }
     const int H = is_q ? p.Hq : p.Hkv;
+    const long long ext = static_cast<long long>(p.B) * rows * H * p.D;
+    if (!in_bounds(row * H * p.D, static_cast<long long>(H) * p.D, ext, p.status)) continue;
     __nv_bfloat16* x = (is_q ? p.q : p.k) + row * H * p.D;
     rotate_row(x, H, p.D, j, c, s);
   }

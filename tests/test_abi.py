@@ -36,6 +36,18 @@ def test_every_declared_symbol_is_exported(lib):
         assert name in _lib.SIGNATURES, name
 
 
+def test_checked_build_exports_the_same_abi():
+    """libhd_checked.so (HD_CHECK_BOUNDS) loads, exports every declared symbol and
+    reports its flag; the normal library reports none."""
+    build(checked=True)
+    checked = _lib.lib_checked()
+    for name in _declared():
+        assert hasattr(checked, name), name
+    assert checked.hd_build_flags() == 1
+    assert hd.lib().hd_build_flags() == 0
+    assert checked.hd_version() == hd.lib().hd_version()
+
+
 def test_version_and_status_strings(lib):
     assert hd.lib().hd_version() >> 16 == 1
     for code in range(6):

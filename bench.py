@@ -1,24 +1,29 @@
 #!/usr/bin/env python
 """Benchmark of the Hidden Decoding hot path on B200 (one JSON line on rank 0).
 
-One step = one pass of every hot-path operation over one batch of synthetic
-input at the intra-stream training workload's sizes (B4, n4, L2048 -> 8192
-expanded positions, 16 query / 4 KV heads, head_dim 128):
-  1. hd_expand_embed   ids [4, 2048] -> X [4, 8192, 2048] from 4 fp32 tables
-  2. hd_attn_fwd + hd_attn_bwd, INTRA
-  3. hd_attn_fwd + hd_attn_bwd, CROSS_FULL
-  4. hd_attn_fwd + hd_attn_bwd, CROSS_WINDOW (W = 1024 tokens = 4096 positions)
-  5. hd_attn_fwd + hd_attn_bwd, final-stream-only queries (KV-mirror), CROSS_FULL
-  6. hd_decode_attn, CROSS_FULL and INTRA, 4 new stream queries per sequence
-     against a 2048-token cache.
+One step = one pass of every hot-path operation, each at its own workload
+configuration's sizes, over synthetic inputs resident in HBM:
+  c2  hd_attn_fwd + hd_attn_bwd, INTRA: B4 n4 L2048 (8192 expanded positions),
+      16 query / 4 KV heads, head_dim 128
+  c3  hd_attn_fwd + hd_attn_bwd, CROSS_WINDOW (W = 1024 tokens = 4096
+      positions): B2 n4 L8192 (32768 positions), 32 / 8 heads
+  c4  hd_attn_fwd, CROSS_FULL over 131072 positions, and final-stream-only
+      queries (KV-mirror, 32768 rows) with their hd_attn_bwd: B1 n4 L32768,
+      32 / 8 heads
+  c5  hd_decode_attn, CROSS_FULL and INTRA, 4 new stream queries per sequence
+      against a 16384-token cache, batch 8 and batch 64
+  x   hd_expand_embed, ids [4, 8192] -> X [4, 32768, 4096] from 4 fp32 tables
 value = unmasked attention TFLOP/s over the step (fwd 4*D, bwd 10*D FLOPs per
-visible (query, key, head) pair, decode 4*D per pair).
+visible (query, key, head) pair, decode 4*D per pair); per_op carries every
+operation's time, TFLOP/s or GB/s and roofline fraction.
 
---workload selects a single-configuration measurement instead: intra_train,
-cross_window, long_cross (fwd/bwd at those sizes), decode8 / decode64 /
-decode8_final (decode steps), expand, rope (RoPE of q and k at 131072
-positions), lm_head and lm_head_train (final-stream LM-head cross-entropy, and
-with its gradients). HBM-bound workloads report GB/s, the rest TFLOP/s.
+--workload selects another measurement: step_intra_train (every row at the
+intra-stream layer's sizes, a 10 ms step), intra_train, cross_window,
+long_cross, long_cross_train (fwd/bwd of one configuration), decode8 /
+decode64 / decode8_final (decode steps), expand, rope (RoPE of q and k at
+131072 positions), lm_head and lm_head_train (final-stream LM-head
+cross-entropy, and with its gradients). HBM-bound workloads report GB/s, the
+rest TFLOP/s.
 
 --impl reference times the float64 CPU oracle (the reference arm) on a bounded
 sample of the same workload. Multi-GPU (torchrun): every rank runs its own
@@ -44,7 +49,23 @@ import torch  # noqa: E402
 
 INTRA, CROSS_FULL, CROSS_WINDOW = 0, 1, 2
 METRIC = "unmasked attention TFLOP/s & expanded tokens/s (fwd+bwd); decode µs/step, GB/s"
-WL = dict(B=4, L=2048, n=4, Hq=16, Hkv=4, D=128, W=1024, V=32000, d=2048, T=2048)
+
+# Sizes of the five workload configurations the hot path is measured on (V and
+# d size the expansion tables; T is the decode cache's prior tokens).
+CFG = {
+    # intra-stream training layer
+    "c2": dict(B=4, L=2048, n=4, Hq=16, Hkv=4, D=128, W=1024, V=32000, d=2048, T=2048),
+    # cross-stream sliding-window layer, window 1024 tokens = 4096 positions
+    "c3": dict(B=2, L=8192, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=8192),
+    # long-context full cross-stream layer (+ final-stream-only queries, KV-mirror)
+    "c4": dict(B=1, L=32768, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=32768),
+    # multi-stream decode step against a 16384-token cache, batch 8 and 64
+    "c5b8": dict(B=8, L=1, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=16384),
+    "c5b64": dict(B=64, L=1, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=16384),
+    # embedding expansion: 4 fp32 tables of 32000 x 4096, 32768 tokens
+    "x": dict(B=4, L=8192, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=1),
+}
+WL = CFG["c2"]
 
 
 # ------------------------------------------------------------------ counting
@@ -112,51 +133,56 @@ def step_plan(wl):
 
 LAUNCHES = {"expand": 1, "fwd": 1, "bwd": 3, "decode": 2, "decode_final": 2, "rope": 1, "lm_head": 2,
             "lm_head_bwd": 3}
-# operations measured on their own only (not part of the default hot-path step)
-EXTRA_KINDS = {"rope", "decode_final", "lm_head", "lm_head_bwd"}
 
-# Extra workloads for per-configuration measurements (`--workload`); the
-# default is the whole hot-path step above.
+# A workload is a list of parts: (label, sizes, operation names of step_plan).
+# The default "step" is one pass of every hot-path row at the configurations'
+# own sizes; the others measure one configuration (or one supplementary kernel).
 WORKLOADS = {
-    "step": dict(WL, ops=None),
-    "intra_train": dict(B=4, L=2048, n=4, Hq=16, Hkv=4, D=128, W=1024, V=32000, d=2048, T=2048,
-                        ops=["fwd_intra", "bwd_intra"]),
-    "cross_window": dict(B=2, L=8192, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=8192,
-                         ops=["fwd_cross_window", "bwd_cross_window"]),
-    "long_cross": dict(B=1, L=32768, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=32768,
-                       ops=["fwd_cross_full", "fwd_final_only"]),
-    "decode8": dict(B=8, L=1, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=16384,
-                    ops=["decode_cross_full", "decode_intra"]),
-    "decode64": dict(B=64, L=1, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=16384,
-                     ops=["decode_cross_full", "decode_intra"]),
-    "expand": dict(B=4, L=8192, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=1,
-                   ops=["expand"]),
-    "decode8_final": dict(B=8, L=1, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=16384,
-                          ops=["decode_final_cross_full", "decode_final_intra"]),
-    "lm_head": dict(B=2, L=8192, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=1,
-                    ops=["lm_head_ce"]),
-    "lm_head_train": dict(B=2, L=8192, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=1,
-                          ops=["lm_head_ce", "lm_head_ce_bwd"]),
-    "rope": dict(B=1, L=32768, n=4, Hq=32, Hkv=8, D=128, W=1024, V=32000, d=4096, T=1,
-                 ops=["rope"]),
+    "step": [("c2", CFG["c2"], ["fwd_intra", "bwd_intra"]),
+             ("c3", CFG["c3"], ["fwd_cross_window", "bwd_cross_window"]),
+             ("c4", CFG["c4"], ["fwd_cross_full", "fwd_final_only", "bwd_final_only"]),
+             ("c5b8", CFG["c5b8"], ["decode_cross_full", "decode_intra"]),
+             ("c5b64", CFG["c5b64"], ["decode_cross_full", "decode_intra"]),
+             ("x", CFG["x"], ["expand"])],
+    # every row at the intra-stream layer's sizes in one short step (decode
+    # against a 2048-token cache)
+    "step_intra_train": [("", CFG["c2"], ["expand", "fwd_intra", "bwd_intra", "fwd_cross_full", "bwd_cross_full",
+                                          "fwd_cross_window", "bwd_cross_window", "fwd_final_only",
+                                          "bwd_final_only", "decode_cross_full", "decode_intra"])],
+    "intra_train": [("", CFG["c2"], ["fwd_intra", "bwd_intra"])],
+    "cross_window": [("", CFG["c3"], ["fwd_cross_window", "bwd_cross_window"])],
+    "long_cross": [("", CFG["c4"], ["fwd_cross_full", "fwd_final_only"])],
+    "long_cross_train": [("", CFG["c4"], ["fwd_final_only", "bwd_final_only"])],
+    "decode8": [("", CFG["c5b8"], ["decode_cross_full", "decode_intra"])],
+    "decode64": [("", CFG["c5b64"], ["decode_cross_full", "decode_intra"])],
+    "decode8_final": [("", CFG["c5b8"], ["decode_final_cross_full", "decode_final_intra"])],
+    "expand": [("", CFG["x"], ["expand"])],
+    "lm_head": [("", dict(CFG["c3"], T=1), ["lm_head_ce"])],
+    "lm_head_train": [("", dict(CFG["c3"], T=1), ["lm_head_ce", "lm_head_ce_bwd"])],
+    "rope": [("", dict(CFG["c4"], T=1), ["rope"])],
 }
 
 
 def plan_for(name):
-    wl = dict(WORKLOADS[name])
-    ops = step_plan(wl)
-    if wl["ops"] is not None:
-        ops = [o for o in ops if o["name"] in wl["ops"]]
-    else:
-        ops = [o for o in ops if o["kind"] not in EXTRA_KINDS]
-    return wl, ops
+    """[(label, sizes, ops)] of a workload; op names get the part's label as prefix."""
+    parts = []
+    for label, wl, names in WORKLOADS[name]:
+        by_name = {o["name"]: o for o in step_plan(dict(wl))}
+        ops = []
+        for nm in names:
+            o = dict(by_name[nm])
+            o["op"] = nm
+            o["name"] = f"{label}.{nm}" if label else nm
+            ops.append(o)
+        parts.append((label, dict(wl), ops))
+    return parts
 
 
 # --------------------------------------------------------------- GPU state
-class Step:
-    """Device buffers of one step plus the calls that make up the step.
+class Part:
+    """Device buffers of one configuration plus the calls of its operations.
 
-    Only the buffers the step's operations use are allocated.
+    Only the buffers its operations use are allocated.
     """
 
     def __init__(self, wl, ops, dev):
@@ -167,24 +193,25 @@ class Step:
         B, n, L, Hq, Hkv, D, V, d, T = (wl[k] for k in ("B", "n", "L", "Hq", "Hkv", "D", "V", "d", "T"))
         S = n * L
         kinds = {o["kind"] for o in ops}
-        names = {o["name"] for o in ops}
         attn = kinds & {"fwd", "bwd"}
         fin = any(o.get("fin") for o in ops if o["kind"] in ("fwd", "bwd"))
         full = any(not o.get("fin") for o in ops if o["kind"] in ("fwd", "bwd"))
+        bwd_fin = any(o.get("fin") for o in ops if o["kind"] == "bwd")
+        bwd_full = any(not o.get("fin") for o in ops if o["kind"] == "bwd")
         # host copies (pinned) of every per-step input, for the end-to-end leg
         self.h = {}
         if "expand" in kinds:
             self.h["ids"] = syn.token_ids(B, L, V, seed=9)
         if attn:
-            a = syn.attention_inputs(B, L, n, Hq, Hkv, D, seed=2, with_grad="bwd" in kinds)
+            a = syn.attention_inputs(B, L, n, Hq, Hkv, D, seed=2, with_grad=bwd_full)
             self.h.update({"k": a["k"], "v": a["v"]})
             if full:
                 self.h["q"] = a["q"]
-                if "bwd" in kinds:
+                if bwd_full:
                     self.h["do"] = a["do"]
             if fin:
                 self.h["qf"] = syn.normal_bf16((B, L, Hq, D), 12)
-                if "bwd" in kinds:
+                if bwd_fin:
                     self.h["dof"] = syn.normal_bf16((B, L, Hq, D), 13)
         if "decode" in kinds:
             self.h["dq_new"] = syn.normal_bf16((B, n, Hq, D), 14)
@@ -239,22 +266,21 @@ class Step:
         self.o, self.lse = {}, {}
         for o in ops:
             if o["kind"] == "fwd":
-                key = o["name"].split("_", 1)[1]
+                key = o["op"].split("_", 1)[1]
                 rows = L if o["fin"] else S
                 self.o[key] = torch.empty((B, rows, Hq, D), dtype=torch.bfloat16, device=dev)
                 self.lse[key] = torch.empty((B, Hq, rows), dtype=torch.float32, device=dev)
         if "bwd" in kinds:
-            if full:
+            if bwd_full:
                 self.dq = torch.empty_like(self.d["q"])
-            if fin:
+            if bwd_fin:
                 self.dqf = torch.empty_like(self.d["qf"])
             self.dk = torch.empty_like(self.d["k"])
             self.dv = torch.empty_like(self.d["v"])
-            self.ws_bwd_n = hd.hd_attn_bwd_workspace_bytes(B, L, n, Hq, Hkv, D, 0 if full else 1)
+            self.ws_bwd_n = hd.hd_attn_bwd_workspace_bytes(B, L, n, Hq, Hkv, D, 0 if bwd_full else 1)
             self.ws_bwd = torch.empty(self.ws_bwd_n, dtype=torch.uint8, device=dev)
-        self.flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
         self.h2d_bytes = sum(t.numel() * t.element_size() for t in self.h.values())
-        # the step's result read back to the host: decode outputs, else the first forward's LSE
+        # the part's result read back to the host: decode outputs, else the first forward's LSE
         self.result = []
         if "decode" in kinds:
             self.result += list(self.dec_o.values())
@@ -272,7 +298,7 @@ class Step:
         self.d2h_bytes = sum(t.numel() * t.element_size() for t in self.results(self.d))
 
     def results(self, d):
-        """The step's result tensors for input set d (read back to the host)."""
+        """The part's result tensors for input set d (read back to the host)."""
         return [d[t][:, :1] if isinstance(t, str) else t for t in self.result]
 
     def call(self, op, stream, d=None):
@@ -281,7 +307,7 @@ class Step:
         B, n, L, Hq, Hkv, D, W, T = (wl[k] for k in ("B", "n", "L", "Hq", "Hkv", "D", "W", "T"))
         sc = 1.0 / math.sqrt(D)
         s = stream.cuda_stream
-        name = op["name"]
+        name = op["op"]
         if op["kind"] == "expand":
             hd.hd_expand_embed(d["ids"], self.tables, self.x, B, L, n, wl["V"], wl["d"], 4, s)
         elif op["kind"] == "lm_head":
@@ -316,14 +342,41 @@ class Step:
                               self.ws_dec, self.ws_dec_n, s)
 
     def h2d(self, d):
-        """Copy the step's inputs from pinned host memory into input set d (current stream)."""
+        """Copy the part's inputs from pinned host memory into input set d (current stream)."""
         for k_, v_ in self.h.items():
             d[k_].copy_(v_, non_blocking=True)
 
     def d2h(self, d):
-        """Copy the step's result back into pinned host memory (current stream)."""
+        """Copy the part's result back into pinned host memory (current stream)."""
         for h_, t_ in zip(self.host_res, self.results(d)):
             h_.copy_(t_, non_blocking=True)
+
+
+class Step:
+    """The parts of a workload and its operations in step order: (part index, op)."""
+
+    def __init__(self, parts, dev):
+        self.parts = [Part(wl, ops, dev) for _, wl, ops in parts]
+        self.ops = [(i, o) for i, (_, _, ops) in enumerate(parts) for o in ops]
+        self.flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        self.h2d_bytes = sum(p.h2d_bytes for p in self.parts)
+        self.d2h_bytes = sum(p.d2h_bytes for p in self.parts)
+
+    def input_sets(self):
+        """The two device input sets, each a list with one dict per part."""
+        return [[p.d for p in self.parts], [p.d_alt for p in self.parts]]
+
+    def call(self, k, stream, dset=None):
+        i, op = self.ops[k]
+        self.parts[i].call(op, stream, None if dset is None else dset[i])
+
+    def h2d(self, dset):
+        for p, d in zip(self.parts, dset):
+            p.h2d(d)
+
+    def d2h(self, dset):
+        for p, d in zip(self.parts, dset):
+            p.d2h(d)
 
 
 # ------------------------------------------------------------------ clocks
@@ -381,35 +434,49 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------- CPU oracle leg
-def oracle_sample(budget_s, wl, seed=0):
+_ORACLE_INPUTS = {}
+
+
+def _oracle_inputs(label, wl):
+    """float64 copies of batch 0 of a configuration's synthetic inputs (cached)."""
+    if label not in _ORACLE_INPUTS:
+        from structured_causal_attention_b200 import synthetic as syn
+
+        B, n, L, Hq, Hkv, D = (wl[k] for k in ("B", "n", "L", "Hq", "Hkv", "D"))
+        a = syn.attention_inputs(1, L, n, Hq, Hkv, D, seed=2)
+        t = {k: a[k].to(torch.float64).numpy() for k in ("q", "k", "v")}
+        t["qf"] = syn.normal_bf16((1, L, Hq, D), 12).to(torch.float64).numpy()
+        _ORACLE_INPUTS[label] = t
+    return _ORACLE_INPUTS[label]
+
+
+def oracle_sample(budget_s, parts, seed=0):
     """Time the float64 oracle on a bounded sample of the step's attention work.
 
-    Returns (unmasked FLOPs done, seconds, description). Query rows are drawn
-    from the four forward operations of the step (INTRA, CROSS_FULL,
-    CROSS_WINDOW, final-stream-only) and credited 4*D FLOPs per visible pair.
+    Returns (unmasked FLOPs done, seconds, description). Each draw takes 32
+    random query rows of one random head of every forward operation of the
+    step, at that operation's own sizes (batch 0), and is credited 4*D FLOPs
+    per visible pair.
     """
     import oracle
-    from structured_causal_attention_b200 import synthetic as syn
 
-    B, n, L, Hq, Hkv, D, W = (wl[k] for k in ("B", "n", "L", "Hq", "Hkv", "D", "W"))
-    S = n * L
     rng = np.random.default_rng(seed)
-    a = syn.attention_inputs(1, L, n, Hq, Hkv, D, seed=2)
-    a64 = {k: a[k].float().numpy().astype(np.float64) for k in ("q", "k", "v")}
-    qf = a64["q"][:, n - 1::n].copy()
-    sc = 1.0 / math.sqrt(D)
-    cases = [(INTRA, 0), (CROSS_FULL, 0), (CROSS_WINDOW, 0), (CROSS_FULL, 1)]
+    cases = [(label, wl, o) for label, wl, ops in parts for o in ops if o["kind"] == "fwd"]
+    for label, wl, _ in cases:
+        _oracle_inputs(label, wl)
     flops, t0, nrows = 0, time.perf_counter(), 0
     while time.perf_counter() - t0 < budget_s:
-        for mode, fin in cases:
+        for label, wl, o in cases:
+            n, L, Hq, D, W = (wl[k] for k in ("n", "L", "Hq", "D", "W"))
+            a64 = _oracle_inputs(label, wl)
+            fin, mode = o["fin"], o["mode"]
             h = int(rng.integers(Hq))
-            Sq = L if fin else S
-            rows = rng.choice(Sq, 32, replace=False)
-            q = qf if fin else a64["q"]
-            oracle.attn_fwd_rows(q, a64["k"], a64["v"], n, mode, W, bool(fin), sc, 0, h, rows)
+            rows = rng.choice(L if fin else n * L, 32, replace=False)
+            q = a64["qf"] if fin else a64["q"]
+            oracle.attn_fwd_rows(q, a64["k"], a64["v"], n, mode, W, bool(fin), 1.0 / math.sqrt(D), 0, h, rows)
             pos = rows * n + (n - 1) if fin else rows
             if mode == INTRA:
-                vis = pos // n + 1
+                vis = (pos // n + 1) if not fin else (rows + 1)
             elif mode == CROSS_FULL:
                 vis = pos + 1
             else:
@@ -417,8 +484,9 @@ def oracle_sample(budget_s, wl, seed=0):
             flops += int(4 * D * vis.sum())
             nrows += len(rows)
     dt = time.perf_counter() - t0
-    return flops, dt, f"{nrows} query rows (32 per draw) of the INTRA, CROSS_FULL, CROSS_WINDOW and " \
-                      f"final-stream-only forward, batch 0, random heads, float64 oracle"
+    names = ", ".join(o["name"] for _, _, o in cases)
+    return flops, dt, f"{nrows} query rows (32 per draw) of the forward operations {names}, batch 0, " \
+                      f"random heads, float64 oracle"
 
 
 def blas_threads():
@@ -448,13 +516,18 @@ def whole_job_value(flops_per_step, world, ms_per_step):
 
 # ------------------------------------------------------------------- main
 DESCRIPTIONS = {
-    "step": "intra_train-sized hot-path step: B4 n4 L2048 (8192 expanded positions), Hq16 Hkv4 D128; "
-            "expand (V32000 d2048 fp32 tables) + fwd/bwd INTRA, CROSS_FULL, CROSS_WINDOW(W=1024 tokens), "
-            "final-stream-only + decode (cache 2048 tokens, CROSS_FULL and INTRA)",
+    "step": "every hot-path row at the configurations' own sizes: c2 INTRA fwd+bwd B4 n4 L2048 Hq16 Hkv4 D128; "
+            "c3 CROSS_WINDOW fwd+bwd B2 n4 L8192 W1024 tokens Hq32 Hkv8; c4 CROSS_FULL fwd (131072 queries) and "
+            "final-stream-only fwd+bwd (32768 queries) B1 n4 L32768 Hq32 Hkv8; c5 decode CROSS_FULL + INTRA, "
+            "16384-token cache, B8 and B64; x expansion B4 L8192 n4 V32000 d4096 fp32",
+    "step_intra_train": "every row at the intra_train sizes: B4 n4 L2048 (8192 expanded positions), Hq16 Hkv4 "
+                        "D128; expand (V32000 d2048 fp32 tables) + fwd/bwd INTRA, CROSS_FULL, CROSS_WINDOW(W=1024 "
+                        "tokens), final-stream-only + decode (cache 2048 tokens, CROSS_FULL and INTRA)",
     "intra_train": "INTRA fwd+bwd, B4 n4 L2048 (8192 expanded), Hq16 Hkv4 D128",
     "cross_window": "CROSS_WINDOW fwd+bwd, B2 n4 L8192 (32768 expanded), W=1024 tokens, Hq32 Hkv8 D128",
     "long_cross": "CROSS_FULL fwd (131072 queries) + final-stream-only fwd (32768 queries), B1 n4 L32768, "
                   "Hq32 Hkv8 D128",
+    "long_cross_train": "final-stream-only fwd+bwd (32768 queries, 131072 keys), B1 n4 L32768, Hq32 Hkv8 D128",
     "decode8": "decode step CROSS_FULL + INTRA, B8 n4, 16384 prior tokens (65540 cache rows), Hq32 Hkv8 D128",
     "decode64": "decode step CROSS_FULL + INTRA, B64 n4, 16384 prior tokens (65540 cache rows), Hq32 Hkv8 D128",
     "expand": "expansion B4 L8192 n4, V32000, d4096 fp32 tables",
@@ -468,13 +541,45 @@ DESCRIPTIONS = {
 }
 
 # DRAM bytes per launch of the dominant kernel from the last ncu capture of
-# the same build (dram__bytes_read.sum + dram__bytes_write.sum); None when the
-# kernel changed after that capture.
+# the same build (dram__bytes_read.sum + dram__bytes_write.sum); a workload
+# whose dominant kernel changed after its capture has no entry (null).
 NCU_TRAFFIC = {
-    ("step", "bwd_cross_full"): 4.810e9,  # attn_bwd_tc_kernel
-    ("lm_head", "lm_head_ce"): 2.280e9,   # lm_head_ce_kernel
-    ("rope", "rope"): 2.628e9,            # rope_kernel
+    ("step_intra_train", "bwd_cross_full"): 4.810e9,  # attn_bwd_tc_kernel
+    ("lm_head", "lm_head_ce"): 2.280e9,               # lm_head_ce_kernel
+    ("rope", "rope"): 2.628e9,                        # rope_kernel
 }
+
+KERNELS = {"fwd": "hd_attn_fwd (attn_fwd_tc_kernel)",
+           "bwd": "hd_attn_bwd (bwd_pre + attn_bwd_tc_kernel + bwd_dq)",
+           "decode": "hd_decode_attn (decode_split + decode_combine)",
+           "expand": "hd_expand_embed (expand_kernel)",
+           "decode_final": "hd_decode_attn_final (decode_split + decode_combine)",
+           "rope": "hd_rope_expanded (rope_kernel)",
+           "lm_head": "hd_lm_head_ce (lm_head_ce_kernel + lm_head_combine)",
+           "lm_head_bwd": "hd_lm_head_ce_bwd (gradient pass + two gemm_tc_kernel)"}
+TENSOR_KINDS = ("fwd", "bwd", "lm_head", "lm_head_bwd")
+HBM_KINDS = ("decode", "decode_final", "expand", "rope")
+
+
+def roofline_of(op, ms, peaks):
+    """Roofline record of one operation from its mean CUDA-event time.
+
+    Tensor-core operations are compared with the measured burst bf16 GEMM
+    rate (frac) and, beside it, with the sustained one (frac_of_sustained);
+    HBM-bound ones with the measured copy bandwidth.
+    """
+    burst = peaks.get("bf16_tflops", 1590.0)
+    sustained = peaks.get("bf16_tflops_sustained", 1400.0)
+    hbm = peaks.get("hbm_gbs", 6650.0)
+    src = "MEASURED_PEAKS.json" if peaks else "fallback"
+    if op["kind"] in TENSOR_KINDS:
+        ach = op["flops"] / (ms * 1e-3) / 1e12
+        return {"bound": "tensor", "achieved": round(ach, 1), "peak": burst, "unit": "TFLOP/s",
+                "frac": round(ach / burst, 4), "peak_source": f"{src} bf16_tflops (burst)",
+                "frac_of_sustained": round(ach / sustained, 4)}
+    ach = op["bytes"] / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s", "frac": round(ach / hbm, 4),
+            "peak_source": f"{src} hbm_gbs"}
 
 
 def main():
@@ -490,13 +595,16 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    wl, ops = plan_for(args.workload)
+    parts = plan_for(args.workload)
+    ops = [o for _, _, pops in parts for o in pops]
     total_flops = sum(o["flops"] for o in ops)
     total_bytes = sum(o.get("bytes", 0) for o in ops)
-    hbm_only = total_flops == 0 or all(o["kind"] in ("decode", "decode_final", "expand", "rope") for o in ops)
-    tokens = wl["B"] * wl["n"] * wl["L"]
+    hbm_only = total_flops == 0 or all(o["kind"] in HBM_KINDS for o in ops)
+    attn_parts = [wl for _, wl, pops in parts if any(o["kind"] in ("fwd", "bwd") for o in pops)]
+    tokens = sum(wl["B"] * wl["n"] * wl["L"] for wl in attn_parts)
+    big = max((wl for _, wl, _ in parts), key=lambda w: w["B"] * w["n"] * w["L"])
     config = {"workload": DESCRIPTIONS[args.workload],
-              "global_batch": wl["B"] * max(world, 1), "seq_len": wl["n"] * wl["L"],
+              "global_batch": big["B"] * max(world, 1), "seq_len": big["n"] * big["L"],
               "parallelism": f"replicas{max(world, 1)}",
               "l2": "256 MB buffer written between timed steps (outside the per-step events); "
                     "per-step working set larger than L2"}
@@ -507,7 +615,7 @@ def main():
         budget = 2.0
         vals = []
         for i in range(args.warmup + args.steps):
-            fl, dt, desc = oracle_sample(budget, WORKLOADS["step"], seed=i)
+            fl, dt, desc = oracle_sample(budget, parts, seed=i)
             if i >= args.warmup:
                 vals.append((fl, dt))
         fl = sum(v[0] for v in vals)
@@ -542,15 +650,15 @@ def main():
     import structured_causal_attention_b200 as hd
 
     hd.lib()
-    st = Step(wl, ops, dev)
+    st = Step(parts, dev)
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
 
-    def one_step(evs=None, d=None):
-        for i, op in enumerate(ops):
+    def one_step(evs=None, dset=None):
+        for i in range(len(st.ops)):
             if evs is not None:
                 evs[i][0].record(stream)
-            st.call(op, stream, d)
+            st.call(i, stream, dset)
             if evs is not None:
                 evs[i][1].record(stream)
 
@@ -590,7 +698,7 @@ def main():
     # training input pipeline does); each step's result is read back after it.
     n_e2e = max(3, args.steps // 2)
     copy_stream = torch.cuda.Stream(device=dev)
-    sets = [st.d, st.d_alt]
+    sets = st.input_sets()
     copied = [torch.cuda.Event(), torch.cuda.Event()]
     consumed = [torch.cuda.Event(), torch.cuda.Event()]
     e_start = torch.cuda.Event(enable_timing=True)
@@ -611,16 +719,15 @@ def main():
                 copied[1 - b].record(copy_stream)
         with torch.cuda.stream(stream):
             stream.wait_event(copied[b])
-            one_step(d=sets[b])
+            one_step(dset=sets[b])
             consumed[b].record(stream)
             st.d2h(sets[b])
     e_end.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = [e_start.elapsed_time(e_end) / n_e2e]
+    e2e_step = e_start.elapsed_time(e_end) / n_e2e
     if hd.hd_device_status() != hd.HD_OK:
         raise RuntimeError("device status set during timing")
 
-    e2e_step = sum(e2e_ms) / len(e2e_ms)
     if world > 1:
         total_ms, e2e_step = reduce_max([total_ms, e2e_step], dev)
     ms_step = total_ms / args.steps
@@ -631,45 +738,27 @@ def main():
             peaks = json.load(f)
     except OSError:
         pass
-    # a kernel timed alone (one-op workloads, tens of ms of load) runs at full clock:
-    # the burst GEMM figure; inside the long multi-op step: the sustained one
-    alone = len(ops) == 1
-    tf_key = "bf16_tflops" if alone else "bf16_tflops_sustained"
-    tf_peak = peaks.get(tf_key, 1590.0 if alone else 1400.0)
-    hbm_peak = peaks.get("hbm_gbs", 6650.0)
     per_op = {}
+    wl_of = {o["name"]: wl for _, wl, pops in parts for o in pops}
     for op, ms in zip(ops, op_ms):
         m = sum(ms) / len(ms)
         rec = {"ms": round(m, 4)}
-        if op["flops"]:
-            rec["tflops"] = round(op["flops"] / (m * 1e-3) / 1e12, 1)
-            if op["kind"] in ("fwd", "bwd", "lm_head", "lm_head_bwd"):
-                rec["frac_of_measured_bf16"] = round(rec["tflops"] / tf_peak, 4)
-        if op.get("bytes"):
-            rec["gbs"] = round(op["bytes"] / (m * 1e-3) / 1e9, 1)
-            rec["frac_of_measured_hbm"] = round(rec["gbs"] / hbm_peak, 4)
+        if op["kind"] in TENSOR_KINDS or op.get("bytes"):
+            r = roofline_of(op, m, peaks)
+            rec["tflops" if r["unit"] == "TFLOP/s" else "gbs"] = r["achieved"]
+            rec["frac"] = r["frac"]
+            if "frac_of_sustained" in r:
+                rec["frac_of_sustained"] = r["frac_of_sustained"]
+        if op["kind"] in ("fwd", "bwd"):
+            wl = wl_of[op["name"]]
+            rows = wl["B"] * wl["L"] * (1 if op["fin"] else wl["n"])
+            rec["query_rows_per_s" if op["fin"] else "expanded_tokens_per_s"] = round(rows / (m * 1e-3), 1)
+        if op["kind"] in ("decode", "decode_final"):
+            rec["us"] = round(1e3 * m, 2)
         per_op[op["name"]] = rec
     dom = max(ops, key=lambda o: per_op[o["name"]]["ms"])
-    dom_ms = per_op[dom["name"]]["ms"]
-    if dom["kind"] in ("fwd", "bwd", "lm_head", "lm_head_bwd"):
-        ach = dom["flops"] / (dom_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": tf_peak, "unit": "TFLOP/s",
-                "frac": round(ach / tf_peak, 4),
-                "peak_source": f"MEASURED_PEAKS.json {tf_key}" if peaks else f"fallback {tf_peak:.0f}"}
-    else:
-        ach = dom["bytes"] / (dom_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak, "unit": "GB/s",
-                "frac": round(ach / hbm_peak, 4),
-                "peak_source": "MEASURED_PEAKS.json hbm_gbs" if peaks else "fallback 6650"}
-    kname = {"fwd": "hd_attn_fwd (attn_fwd_tc_kernel)",
-             "bwd": "hd_attn_bwd (bwd_pre + attn_bwd_tc_kernel + bwd_dq)",
-             "decode": "hd_decode_attn (decode_split + decode_combine)",
-             "expand": "hd_expand_embed (expand_kernel)",
-             "decode_final": "hd_decode_attn_final (decode_split + decode_combine)",
-             "rope": "hd_rope_expanded (rope_kernel)",
-             "lm_head": "hd_lm_head_ce (lm_head_ce_kernel + lm_head_combine)",
-             "lm_head_bwd": "hd_lm_head_ce_bwd (gradient pass + two gemm_tc_kernel)"}[dom["kind"]]
-    roof = {"kernel": f"{kname}, op {dom['name']}", **roof,
+    roof = roofline_of(dom, per_op[dom["name"]]["ms"], peaks)
+    roof = {"kernel": f"{KERNELS[dom['kind']]}, op {dom['name']}", **roof,
             "traffic": NCU_TRAFFIC.get((args.workload, dom["name"]))}
     if hbm_only:
         value = total_bytes * max(world, 1) / (ms_step * 1e-3) / 1e9
@@ -696,12 +785,12 @@ def main():
     }
     if tokens and not hbm_only:
         out["expanded_tokens_per_s"] = round(tokens * max(world, 1) / (ms_step * 1e-3), 1)
-    dec = per_op.get("decode_cross_full")
+    dec = next((per_op[o["name"]] for o in ops if o["kind"] == "decode" and o["mode"] == CROSS_FULL), None)
     if dec:
-        out["decode_us_per_step"] = round(1e3 * dec["ms"], 2)
+        out["decode_us_per_step"] = dec["us"]
         out["decode_gbs"] = dec.get("gbs")
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        fl, dt, desc = oracle_sample(10.0, WORKLOADS["step"])
+        fl, dt, desc = oracle_sample(10.0, parts)
         out["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
                                "kind": "oracle", "sample": f"{dt:.1f} s: " + desc}
     if world > 1:

@@ -45,6 +45,33 @@ def test_step_plan_covers_every_hot_path_row():
     assert fwd["flops"] == 4 * 128 * fwd["pairs"]
 
 
+def test_default_step_runs_every_configuration_at_its_sizes():
+    parts = bench.plan_for("step")
+    names = {o["name"] for _, _, ops in parts for o in ops}
+    assert {"c2.fwd_intra", "c2.bwd_intra", "c3.fwd_cross_window", "c3.bwd_cross_window",
+            "c4.fwd_cross_full", "c4.fwd_final_only", "c4.bwd_final_only", "c5b8.decode_cross_full",
+            "c5b8.decode_intra", "c5b64.decode_cross_full", "c5b64.decode_intra", "x.expand"} == names
+    sizes = {label: wl for label, wl, _ in parts}
+    assert (sizes["c2"]["B"], sizes["c2"]["L"], sizes["c2"]["Hq"], sizes["c2"]["Hkv"]) == (4, 2048, 16, 4)
+    assert (sizes["c3"]["B"], sizes["c3"]["L"], sizes["c3"]["W"], sizes["c3"]["Hq"]) == (2, 8192, 1024, 32)
+    assert (sizes["c4"]["B"], sizes["c4"]["n"] * sizes["c4"]["L"]) == (1, 131072)
+    assert (sizes["c5b8"]["B"], sizes["c5b64"]["B"], sizes["c5b8"]["T"]) == (8, 64, 16384)
+    op = {o["name"]: o for _, _, ops in parts for o in ops}
+    # 4a: 131072 (131072 + 1) / 2 pairs per head, 32 heads, 4 * D FLOPs each (BASELINE: 140.7 TFLOP)
+    assert op["c4.fwd_cross_full"]["flops"] == 4 * 128 * 32 * 131072 * 131073 // 2
+    assert abs(op["c4.fwd_cross_full"]["flops"] / 1e12 - 140.7) < 0.1
+    # decode B8: K and V of 65540 cache rows, 8 heads, D128, bf16 (2.148 GB)
+    assert abs(op["c5b8.decode_cross_full"]["bytes"] / 1e9 - 2.148) < 0.01
+
+
+def test_roofline_fraction_uses_the_burst_peak():
+    op = dict(kind="fwd", flops=2e12)
+    r = bench.roofline_of(op, 2.0, {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0})
+    assert r["achieved"] == 1000.0 and r["frac"] == 0.625 and r["frac_of_sustained"] == round(1000 / 1400, 4)
+    d = bench.roofline_of(dict(kind="decode", bytes=6e9), 1.0, {"hbm_gbs": 6000.0})
+    assert d["bound"] == "hbm" and d["frac"] == 1.0
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))

@@ -44,6 +44,18 @@ int check_attn(const void* q, const void* k, const void* v, int B, int L, int n,
   return HD_OK;
 }
 
+// Streaming multiprocessors of the current device; 148 (a B200) when no device
+// can be queried, so that workspace sizes can still be computed without one.
+int sm_count() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) {
+    cudaGetLastError();  // clear the error the failed query recorded
+    return 148;
+  }
+  return sms;
+}
+
 AttnParams make_params(const void* q, const void* k, const void* v, int B, int L, int n, int Hq,
                        int Hkv, int D, int mode, int W, int final_only, float scale) {
   AttnParams p = {};
@@ -111,17 +123,6 @@ size_t packed_rows(int B, int L, int n, int Hq, int final_only) {
 
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? HD_OK : HD_ERR_CUDA; }
 
-// Streaming multiprocessors of the current device; 148 (a B200) when no device
-// can be queried, so that workspace sizes can still be computed without one.
-int sm_count() {
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) {
-    cudaGetLastError();  // clear the error the failed query recorded
-    return 148;
-  }
-  return sms;
-}
 
 // Split-K partials for `rows` query rows per (sequence, KV head) against up to
 // `keys` keys: unnormalised O (fp32 [.., D]) and (max, sum) pairs.

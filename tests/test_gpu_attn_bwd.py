@@ -98,7 +98,7 @@ def _sampled(name, mode, seed, qpairs, kvpairs, rows_per_head=256, final_only=Fa
     closed form sum_keys dV = sum over the group's query heads and rows of dO
     (each row's P sums to one)."""
     need_gpu()
-    w = syn.WORKLOADS[name]
+    w = syn.WORKLOADS[name] if isinstance(name, str) else name
     B, L, n, Hq, Hkv, D = w["B"], w["L"], w["n"], w["Hq"], w["Hkv"], w["D"]
     W = w.get("W", 0)
     inp = syn.attention_inputs(B, L, n, Hq, Hkv, D, final_only=final_only, seed=seed, with_grad=True)
@@ -177,3 +177,19 @@ def test_bwd_long_cross_final_only_workload_sampled():
         return np.unique(np.concatenate([np.arange(s0, s0 + 64) for s0 in st]))
 
     _sampled("long_cross", hd.CROSS_FULL, 8, qpairs, [(0, 0), (0, 5)], final_only=True, key_starts=starts)
+
+
+def test_bwd_long_problem_partial_bucket_sampled():
+    """A causal problem of 516 key tiles (66000 positions): the grid buckets 64
+    key tiles of one (batch, KV head) together when a problem has at least 512,
+    so here 8 full buckets and a partial one of 4 tiles. dQ on 256 rows per
+    head; dK/dV on runs in the partial bucket, across its start (key 65536) and
+    at the end."""
+    w = dict(B=1, L=16500, n=4, Hq=2, Hkv=1, D=64, scale=0.125)
+    S = w["n"] * w["L"]
+
+    def starts(b, kh):
+        st = [S - 64, 65536 - 32, 65536 + 200, S - 300]
+        return np.unique(np.concatenate([np.arange(s0, s0 + 64) for s0 in st]))
+
+    _sampled(w, hd.CROSS_FULL, 9, [(0, 0), (0, 1)], [(0, 0)], key_starts=starts)

@@ -84,6 +84,18 @@ __host__ __device__ __forceinline__ bool fwd_head_pairs(const AttnParams& p) {
   return (p.Hq / p.Hkv) % 2 == 0;
 }
 
+// Grid order of head-paired CTAs. Query-tile-major (the heaviest tiles of
+// every problem first) balances short problems. For long full-causal ones
+// (no window, one stream group, at least 128 query tiles) it spreads the
+// CTAs running at once over every KV head, so each head's K/V tiles are read
+// by CTAs far apart in time and come back from DRAM: 203 GB of DRAM reads
+// for one forward at 131072 positions, whose algorithmic bytes are 2.7 GB.
+// Those problems take a KV-head-major order instead: 3.2 GB of reads, an L2
+// hit rate of 99 % against 39 %, and 6 % less time at the power cap.
+__host__ __device__ __forceinline__ bool fwd_kv_major(const AttnParams& p, int num_qt) {
+  return p.win >= p.Lk && p.groups == 1 && num_qt >= 128;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ,
@@ -107,7 +119,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int num_qt = (p.Lq + kBM - 1) / kBM;
   const bool head_pair = fwd_head_pairs(p);
   int b, grp, h0, h1, r00, r01;  // batch, stream group; head and first row of tile 0 / 1
-  if (head_pair) {
+  if (head_pair && fwd_kv_major(p, num_qt)) {
+    // long full-causal problems: every CTA of one (batch, KV head) before the
+    // next one's, heaviest query tiles first inside it, so the CTAs running at
+    // once read the same KV head's tiles and keep them in L2
+    const int pairs = p.Hq / p.Hkv / 2;  // head pairs per KV head
+    const int per_kv = num_qt * pairs;
+    const int bk = static_cast<int>(blockIdx.x / per_kv);
+    const int rem = static_cast<int>(blockIdx.x % per_kv);
+    const int qt = num_qt - 1 - rem / pairs;
+    grp = 0;
+    b = bk / p.Hkv;
+    h0 = 2 * ((bk % p.Hkv) * pairs + rem % pairs);
+    h1 = h0 + 1;
+    r00 = r01 = qt * kBM;
+  } else if (head_pair) {
     // the same 128 rows of two query heads that share a KV head: both tiles
     // visit exactly the same K/V tiles
     const int bhg = p.B * (p.Hq / 2) * p.groups;

@@ -47,8 +47,8 @@ constexpr int kKN = 128;   // keys per CTA
 constexpr int kQM = 64;    // query rows per iteration
 constexpr int kQS = 3;     // Q / dO stages
 constexpr int kThreads = 480;
-constexpr int kKB = 8;       // key tiles per grid bucket (INTRA, short windows)
-constexpr int kKBLong = 64;  // key tiles per grid bucket (long causal problems)
+constexpr int kKB = 8;         // key tiles per grid bucket (INTRA, short windows)
+constexpr int kLongKT = 512;   // a problem this many key tiles long is one bucket
 constexpr uint32_t kTmemCols = 512;
 
 template <int D>
@@ -115,16 +115,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Inside a bucket a problem's key tiles are adjacent, so they run at the
   // same time and share their Q, dO and dQ tiles in L2. Buckets of kKB key
   // tiles for INTRA problems (one stream each, many of them) and for windows
-  // short against the sequence (key tiles of nearly equal work). Problems of
-  // at least 8 * kKBLong key tiles take buckets of kKBLong: a wave then holds
-  // the key tiles of two or three problems instead of a slice of every one,
-  // and walks fewer query tiles (the KV-mirror backward at 131072 keys: 4.9 %
-  // faster). Other problems take one key tile per bucket (key-tile-major),
-  // which measured best there.
+  // short against the sequence (key tiles of nearly equal work). A problem of
+  // at least kLongKT key tiles is one bucket: the CTAs running at once then
+  // hold one problem's key tiles instead of a slice of every problem, and walk
+  // its query tiles together (the KV-mirror backward at 131072 keys: 5 %
+  // faster than key-tile-major, DRAM traffic 23.5 -> 6.6 GB). Other problems
+  // take one key tile per bucket (key-tile-major), which measured best there.
   const int bkg = p.B * p.Hkv * p.groups;
   const int num_kt = (p.Lk + kKN - 1) / kKN;
   const bool bucketed = p.groups > 1 || 4LL * p.win <= p.Lk;
-  const int kb = bucketed ? min(kKB, num_kt) : (num_kt >= 8 * kKBLong ? kKBLong : 1);
+  const int kb = bucketed ? min(kKB, num_kt) : (num_kt >= kLongKT ? num_kt : 1);
   const int bucket = static_cast<int>(blockIdx.x / (bkg * kb));
   const int rem = static_cast<int>(blockIdx.x - static_cast<long long>(bucket) * bkg * kb);
   const int bsize = min(kb, num_kt - bucket * kb);

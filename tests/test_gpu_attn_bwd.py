@@ -179,12 +179,11 @@ def test_bwd_long_cross_final_only_workload_sampled():
     _sampled("long_cross", hd.CROSS_FULL, 8, qpairs, [(0, 0), (0, 5)], final_only=True, key_starts=starts)
 
 
-def test_bwd_long_problem_partial_bucket_sampled():
-    """A causal problem of 516 key tiles (66000 positions): the grid buckets 64
-    key tiles of one (batch, KV head) together when a problem has at least 512,
-    so here 8 full buckets and a partial one of 4 tiles. dQ on 256 rows per
-    head; dK/dV on runs in the partial bucket, across its start (key 65536) and
-    at the end."""
+def test_bwd_long_problem_one_bucket_sampled():
+    """A causal problem of 516 key tiles (66000 positions, a tile count that is
+    no power of two): the grid makes a problem of at least 512 key tiles one
+    bucket, its key tiles adjacent, heaviest first. dQ on 256 rows per head;
+    dK/dV on runs at the last tiles, across key 65536 and at the end."""
     w = dict(B=1, L=16500, n=4, Hq=2, Hkv=1, D=64, scale=0.125)
     S = w["n"] * w["L"]
 

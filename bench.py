@@ -546,6 +546,9 @@ DESCRIPTIONS = {
 NCU_TRAFFIC = {
     ("step", "c4.fwd_cross_full"): 4.25e9,            # attn_fwd_tc_kernel (--workload long_cross)
     ("long_cross", "fwd_cross_full"): 4.25e9,         # attn_fwd_tc_kernel
+    ("long_cross_train", "bwd_final_only"): 6.59e9,   # attn_bwd_tc_kernel
+    ("cross_window", "bwd_cross_window"): 20.01e9,    # attn_bwd_tc_kernel
+    ("step_intra_train", "bwd_cross_full"): 3.89e9,   # attn_bwd_tc_kernel
     ("lm_head", "lm_head_ce"): 2.280e9,               # lm_head_ce_kernel
     ("rope", "rope"): 2.628e9,                        # rope_kernel
 }

@@ -324,13 +324,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       };
-      // P of 32 keys -> 16 TMEM columns
+      // P of 32 keys -> 16 TMEM columns. The exponent s*scale*log2(e) - m of a
+      // pair of keys is one paired fp32 FMA (fma.rn.f32x2: each half rounds
+      // like fmaf), which frees issue slots for the exponentials: 4-6 %
+      // faster at the power cap than one fmaf per key.
       auto exp32 = [&](const uint32_t* v, uint32_t col, float m_use) {
         uint32_t pk[16];
+        const uint64_t sc2 = pack_f32x2(p.scale_log2, p.scale_log2);
+        const uint64_t nm2 = pack_f32x2(-m_use, -m_use);
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(v[e]), p.scale_log2, -m_use));
-          const float p1 = fast_exp2(fmaf(__uint_as_float(v[e + 1]), p.scale_log2, -m_use));
+          float x0, x1;
+          fma_f32x2(v[e], v[e + 1], sc2, nm2, x0, x1);
+          const float p0 = fast_exp2(x0);
+          const float p1 = fast_exp2(x1);
           l_run += p0 + p1;
           pk[e >> 1] = pack_bf16(p0, p1);
         }

@@ -132,6 +132,24 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Two fp32 values as one 64-bit register pair (low half first).
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+// (y0, y1) = (a0, a1) * b + c on both halves of a register pair with one
+// paired FMA (sm_100 fma.rn.f32x2); each half rounds exactly like fmaf. a0
+// and a1 are fp32 bit patterns.
+__device__ __forceinline__ void fma_f32x2(uint32_t a0, uint32_t a1, uint64_t b, uint64_t c, float& y0,
+                                          float& y1) {
+  uint64_t a, y;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "r"(a0), "r"(a1));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(y) : "l"(a), "l"(b), "l"(c));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(y0), "=f"(y1) : "l"(y));
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));

@@ -7,7 +7,9 @@ being performed. Each workload configuration runs here at the size the bench
 times, through both builds on the same inputs. The checked build's status word
 must stay HD_OK, so no index left its buffer at any of these sizes, and its
 outputs must equal the normal build's bit for bit: the checks add branches,
-not arithmetic.
+not arithmetic. The one exception is dQ, which many CTAs add into an fp32
+accumulator in an order that differs from run to run (even for one build);
+after the bf16 rounding two runs differ there by at most one bf16 step.
 """
 import ctypes
 import math
@@ -41,16 +43,27 @@ def _gen(shape, seed, dtype=torch.bfloat16):
     return torch.randn(shape, device="cuda", generator=g).to(dtype)
 
 
-def _both(libs, fn):
-    """fn(L) -> tuple of output tensors; run through both builds and compare."""
+def _both(libs, fn, summed=()):
+    """fn(L) -> tuple of output tensors; run through both builds and compare.
+
+    Outputs whose index is in ``summed`` are sums in a run-dependent order:
+    they must agree within one bf16 step (2^-7 of the value, plus 1e-6 for
+    values that cancel to near zero); all others bit for bit.
+    """
     outs = []
     for L in libs:
         outs.append(fn(L))
         torch.cuda.synchronize()
         st = L.hd_device_status(_stream(), 1)
         assert st == hd.HD_OK, hd.status_string(st)
-    for a, b in zip(*outs):
-        assert torch.equal(a, b), "the checked build changed an output"
+    for i, (a, b) in enumerate(zip(*outs)):
+        if i in summed:
+            a32, b32 = a.float(), b.float()
+            tol = 2.0 ** -7 * torch.maximum(a32.abs(), b32.abs()) + 1e-6
+            assert ((a32 - b32).abs() <= tol).all(), \
+                "the checked build changed a summed output by more than one bf16 step"
+        else:
+            assert torch.equal(a, b), "the checked build changed an output"
 
 
 ATTN = [  # name, B, L, n, Hq, Hkv, D, mode, W, final_only, backward
@@ -85,7 +98,7 @@ def test_attention_checked_build_full_size(libs, cfg):
                               mode, W, fin, ctypes.c_float(sc), ws.data_ptr(), wsn, _stream()) == hd.HD_OK
         return out, lse, dq, dk, dv
 
-    _both(libs, run)
+    _both(libs, run, summed=(2,))
 
 
 @pytest.mark.parametrize("B", [8, 64])

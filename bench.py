@@ -19,7 +19,8 @@ operation's time, TFLOP/s or GB/s and roofline fraction.
 
 --workload selects another measurement: step_intra_train (every row at the
 intra-stream layer's sizes, a 10 ms step), intra_train, cross_window,
-long_cross, long_cross_train (fwd/bwd of one configuration), decode8 /
+long_cross, long_cross_train (fwd/bwd of one configuration), cross_full_32k
+(CROSS_FULL fwd+bwd over 32768 positions), decode8 /
 decode64 / decode8_final (decode steps), expand, rope (RoPE of q and k at
 131072 positions), lm_head and lm_head_train (final-stream LM-head
 cross-entropy, and with its gradients). HBM-bound workloads report GB/s, the
@@ -156,6 +157,9 @@ WORKLOADS = {
     "cross_window": [("", CFG["c3"], ["fwd_cross_window", "bwd_cross_window"])],
     "long_cross": [("", CFG["c4"], ["fwd_cross_full", "fwd_final_only"])],
     "long_cross_train": [("", CFG["c4"], ["fwd_final_only", "bwd_final_only"])],
+    # a mid-size full-causal layer (the long-problem grid orders, ~1 GB on the
+    # device): the case the detailed profiles of the long kernels are taken on
+    "cross_full_32k": [("", dict(CFG["c4"], L=8192, T=8192), ["fwd_cross_full", "bwd_cross_full"])],
     "decode8": [("", CFG["c5b8"], ["decode_cross_full", "decode_intra"])],
     "decode64": [("", CFG["c5b64"], ["decode_cross_full", "decode_intra"])],
     "decode8_final": [("", CFG["c5b8"], ["decode_final_cross_full", "decode_final_intra"])],
@@ -531,6 +535,7 @@ DESCRIPTIONS = {
     "long_cross": "CROSS_FULL fwd (131072 queries) + final-stream-only fwd (32768 queries), B1 n4 L32768, "
                   "Hq32 Hkv8 D128",
     "long_cross_train": "final-stream-only fwd+bwd (32768 queries, 131072 keys), B1 n4 L32768, Hq32 Hkv8 D128",
+    "cross_full_32k": "CROSS_FULL fwd+bwd, B1 n4 L8192 (32768 expanded), Hq32 Hkv8 D128",
     "decode8": "decode step CROSS_FULL + INTRA, B8 n4, 16384 prior tokens (65540 cache rows), Hq32 Hkv8 D128",
     "decode64": "decode step CROSS_FULL + INTRA, B64 n4, 16384 prior tokens (65540 cache rows), Hq32 Hkv8 D128",
     "expand": "expansion B4 L8192 n4, V32000, d4096 fp32 tables",

@@ -10,15 +10,17 @@
 // keys. Per query tile, on the tensor cores (one issuing thread, fp32 in TMEM):
 //   S^T  = K Q^T      (M 128 keys, N 64 queries)   } double-buffered in TMEM
 //   dP^T = V dO^T     (M 128 keys, N 64 queries)   }
-//   dV  += P^T dO     (M 128 keys, N D)            } accumulated in TMEM across
+//   dV  += P^T dO     (M 128 keys, N D; P^T in TMEM) } accumulated in TMEM across
 //   dK  += dS^T Q     (M 128 keys, N D)            } the whole group
 //   dQ^T = K^T dS^T   (M D, N 64 queries)           into the S^T buffer
 // Roles (15 warps):
 //   warps 0-7   two warpgroups, one key row per thread, each taking 32 of the
-//               64 query columns: P^T = exp2(S^T - LSE), dS^T = P^T (dP^T - D),
-//               written as bf16 into shared memory in the MMA operand layout;
-//               at the end warpgroup 0 stores dK (scaled) and warpgroup 1 dV
-//               through TMA.
+//               64 query columns: P^T = exp2(S^T - LSE), dS^T = P^T (dP^T - D).
+//               P^T goes as bf16 pairs into TMEM, over the warpgroup's own S^T
+//               columns once they are read (the A operand of dV); dS^T goes
+//               into shared memory in the MMA operand layout (the A operand of
+//               dK, the B operand of dQ^T). At the end warpgroup 0 stores dK
+//               (scaled) and warpgroup 1 dV through TMA.
 //   warps 8-11  one head-dim row per thread: dQ^T from TMEM into an fp32 tile
 //               in shared memory, added into the fp32 dQ accumulator by a TMA
 //               bulk reduce-add (the TMA unit does the adds, not the SM).
@@ -60,8 +62,7 @@ struct BtSmem {
   static constexpr int V_OFF = K_OFF + NSUB * KSUB;
   static constexpr int Q_OFF = V_OFF + NSUB * KSUB;          // kQS stages
   static constexpr int DO_OFF = Q_OFF + kQS * NSUB * QSUB;   // kQS stages
-  static constexpr int P_OFF = DO_OFF + kQS * NSUB * QSUB;   // [128 keys][64 q] bf16
-  static constexpr int DS_OFF = P_OFF + kKN * 128;
+  static constexpr int DS_OFF = DO_OFF + kQS * NSUB * QSUB;  // [128 keys][64 q] bf16
   static constexpr int DQ_OFF = DS_OFF + kKN * 128;          // D/32 boxes of [64 q][32] fp32
   static constexpr int L_OFF = DQ_OFF + (D / 32) * kQM * 32 * 4;  // kQS stages x 64 LSE (log2)
   static constexpr int DL_OFF = L_OFF + kQS * kQM * 4;            // kQS stages x 64 D
@@ -82,7 +83,7 @@ enum {
   B_QE = 4,   // [kQS] stage free (one MMA commit from each issuer)
   B_SF = 7,   // [2] S^T / dP^T ready (MMA commit)
   B_PF = 9,   // P^T / dS^T written (8 warp arrivals)
-  B_PE = 10,  // P^T / dS^T consumed by the MMAs (MMA commit)
+  B_PE = 10,  // dS^T consumed by the MMAs (MMA commit)
   B_DF = 11,  // [2] dQ^T ready (MMA commit)
   B_DE = 13,  // [2] dQ^T read out (4 warp arrivals)
   B_END = 15  // every MMA done (MMA commit)
@@ -100,8 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
   const uint32_t sK = sbase + SM::K_OFF, sV = sbase + SM::V_OFF, sQ = sbase + SM::Q_OFF,
-                 sDO = sbase + SM::DO_OFF, sP = sbase + SM::P_OFF, sDS = sbase + SM::DS_OFF,
-                 sDQ = sbase + SM::DQ_OFF;
+                 sDO = sbase + SM::DO_OFF, sDS = sbase + SM::DS_OFF, sDQ = sbase + SM::DQ_OFF;
   float* sL = reinterpret_cast<float*>(sgen + SM::L_OFF);
   float* sDl = reinterpret_cast<float*>(sgen + SM::DL_OFF);
   auto bar = [&](int i) { return sbase + SM::BAR_OFF + 8u * i; };
@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dK = tc::smem_desc_sw128(sK, 16, 1024), dV = tc::smem_desc_sw128(sV, 16, 1024);
       const uint64_t dQk = tc::smem_desc_sw128(sQ, 16, 1024), dOk = tc::smem_desc_sw128(sDO, 16, 1024);
       const uint64_t dQm = tc::smem_desc_sw128(sQ, SM::QSUB, 1024), dOm = tc::smem_desc_sw128(sDO, SM::QSUB, 1024);
-      const uint64_t dP = tc::smem_desc_sw128(sP, 16, 1024), dS = tc::smem_desc_sw128(sDS, 16, 1024);
+      const uint64_t dS = tc::smem_desc_sw128(sDS, 16, 1024);
       const uint64_t dSm = tc::smem_desc_sw128(sDS, SM::QSUB, 1024);
       const uint64_t dKt = tc::smem_desc_sw128(sK, kt_lbo, 1024);
       auto add = [](uint64_t d, uint32_t bytes) { return d + (bytes >> 4); };
@@ -254,11 +254,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t acc = it > 0 ? 1u : 0u;
 #pragma unroll
           for (int kk = 0; kk < kQM / 16; ++kk) {  // reduce over the 64 queries
-            const uint64_t ap = add(dP, kk * 32);
+            // P^T of queries 16kk..16kk+15: warpgroup kk/2 wrote its 32
+            // queries at S^T columns 32*(kk/2)..+15 of buffer x, two per column
+            const uint32_t ap = tmem + 128 * x + (kk >> 1) * 32 + (kk & 1) * 8;
             const uint64_t as = add(dS, kk * 32);
             const uint64_t bo = add(dOm, st * NSUB * SM::QSUB + kk * 2048);
             const uint64_t bq = add(dQm, st * NSUB * SM::QSUB + kk * 2048);
-            tc::mma_ss_elect(tdV, ap, bo, idKV, (acc | kk) ? 1u : 0u);
+            tc::mma_ts_elect(tdV, ap, bo, idKV, (acc | kk) ? 1u : 0u);
             tc::mma_ss_elect(tdK, as, bq, idKV, (acc | kk) ? 1u : 0u);
           }
 #pragma unroll
@@ -335,7 +337,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           dd[j / 2 + 1] = pack_bf16(dj[2], dj[3]);
         }
       }
-      // the MMAs of the previous tile have finished reading P^T / dS^T
+      // P^T into TMEM over this warpgroup's own S^T columns, read above. Those
+      // columns next take this tile's dQ^T, which the MMAs write only after
+      // dV has read P^T: MMAs from one thread execute in order.
+      tc::tmem_st16(tmem + tq + 128 * x + sw * 32, pp);
+      // the MMAs of the previous tile have finished reading dS^T
       if (it > 0) {
         if (!tc::mbar_wait(bar(B_PE), (it - 1) & 1, abort_flag, p.status)) { ok = false; break; }
       }
@@ -343,13 +349,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int k = 0; k < 4; ++k) {
         const int ch = sw * 4 + k;
         const uint32_t off = row * 128 + ((ch ^ (row & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(sP + off), "r"(pp[4 * k]),
-                     "r"(pp[4 * k + 1]), "r"(pp[4 * k + 2]), "r"(pp[4 * k + 3])
-                     : "memory");
         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(sDS + off), "r"(dd[4 * k]),
                      "r"(dd[4 * k + 1]), "r"(dd[4 * k + 2]), "r"(dd[4 * k + 3])
                      : "memory");
       }
+      tc::tmem_wait_st();
       tc::fence_async_smem();
       tc::tc_fence_before();
       __syncwarp();

@@ -11,16 +11,16 @@
 //   S^T  = K Q^T      (M 128 keys, N 64 queries)   } double-buffered in TMEM
 //   dP^T = V dO^T     (M 128 keys, N 64 queries)   }
 //   dV  += P^T dO     (M 128 keys, N D; P^T in TMEM) } accumulated in TMEM across
-//   dK  += dS^T Q     (M 128 keys, N D)            } the whole group
+//   dK  += dS^T Q     (M 128 keys, N D; dS^T in TMEM) } the whole group
 //   dQ^T = K^T dS^T   (M D, N 64 queries)           into the S^T buffer
 // Roles (15 warps):
 //   warps 0-7   two warpgroups, one key row per thread, each taking 32 of the
 //               64 query columns: P^T = exp2(S^T - LSE), dS^T = P^T (dP^T - D).
-//               P^T goes as bf16 pairs into TMEM, over the warpgroup's own S^T
-//               columns once they are read (the A operand of dV); dS^T goes
-//               into shared memory in the MMA operand layout (the A operand of
-//               dK, the B operand of dQ^T). At the end warpgroup 0 stores dK
-//               (scaled) and warpgroup 1 dV through TMA.
+//               P^T and dS^T go as bf16 pairs into TMEM, over the warpgroup's
+//               own S^T and dP^T columns once they are read (the A operands of
+//               dV and dK), and dS^T also into shared memory in the MMA operand
+//               layout (the B operand of dQ^T). At the end warpgroup 0 stores
+//               dK (scaled) and warpgroup 1 dV through TMA.
 //   warps 8-11  one head-dim row per thread: dQ^T from TMEM into an fp32 tile
 //               in shared memory, added into the fp32 dQ accumulator by a TMA
 //               bulk reduce-add (the TMA unit does the adds, not the SM).
@@ -83,7 +83,7 @@ enum {
   B_QE = 4,   // [kQS] stage free (one MMA commit from each issuer)
   B_SF = 7,   // [2] S^T / dP^T ready (MMA commit)
   B_PF = 9,   // P^T / dS^T written (8 warp arrivals)
-  B_PE = 10,  // dS^T consumed by the MMAs (MMA commit)
+  B_PE = 10,  // dS^T in shared memory consumed by the MMAs (MMA commit)
   B_DF = 11,  // [2] dQ^T ready (MMA commit)
   B_DE = 13,  // [2] dQ^T read out (4 warp arrivals)
   B_END = 15  // every MMA done (MMA commit)
@@ -256,12 +256,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < kQM / 16; ++kk) {  // reduce over the 64 queries
             // P^T of queries 16kk..16kk+15: warpgroup kk/2 wrote its 32
             // queries at S^T columns 32*(kk/2)..+15 of buffer x, two per column
+            // (dS^T likewise at the dP^T columns, 64 further on)
             const uint32_t ap = tmem + 128 * x + (kk >> 1) * 32 + (kk & 1) * 8;
-            const uint64_t as = add(dS, kk * 32);
             const uint64_t bo = add(dOm, st * NSUB * SM::QSUB + kk * 2048);
             const uint64_t bq = add(dQm, st * NSUB * SM::QSUB + kk * 2048);
             tc::mma_ts_elect(tdV, ap, bo, idKV, (acc | kk) ? 1u : 0u);
-            tc::mma_ss_elect(tdK, as, bq, idKV, (acc | kk) ? 1u : 0u);
+            tc::mma_ts_elect(tdK, ap + 64, bq, idKV, (acc | kk) ? 1u : 0u);
           }
 #pragma unroll
           for (int kk = 0; kk < kKN / 16; ++kk) {  // reduce over the 128 keys
@@ -337,10 +337,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           dd[j / 2 + 1] = pack_bf16(dj[2], dj[3]);
         }
       }
-      // P^T into TMEM over this warpgroup's own S^T columns, read above. Those
-      // columns next take this tile's dQ^T, which the MMAs write only after
-      // dV has read P^T: MMAs from one thread execute in order.
+      // P^T and dS^T into TMEM over this warpgroup's own S^T and dP^T columns,
+      // read above. The S^T columns next take this tile's dQ^T, which the MMAs
+      // write only after dV has read P^T: MMAs from one thread execute in
+      // order. (Shared-memory operands cost bandwidth the MMAs need: each of
+      // these moves was 1-2 % faster.)
       tc::tmem_st16(tmem + tq + 128 * x + sw * 32, pp);
+      tc::tmem_st16(tmem + tq + 128 * x + 64 + sw * 32, dd);
       // the MMAs of the previous tile have finished reading dS^T
       if (it > 0) {
         if (!tc::mbar_wait(bar(B_PE), (it - 1) & 1, abort_flag, p.status)) { ok = false; break; }

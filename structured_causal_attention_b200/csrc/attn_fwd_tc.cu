@@ -8,33 +8,34 @@
 // section "隐式序列缩放的技术细节" step 2 (causal attention over the expanded
 // sequence).
 //
-// One CTA = two 128-row query tiles that share every K/V tile the CTA loads:
-// the same rows of two query heads of one GQA group (when the group size is
-// even), so both tiles take exactly the same K/V steps; otherwise two
-// consecutive row tiles of one head. Always of one (batch, stream group).
-//   warps 0-3 / 4-7  softmax warpgroup of query tile 0 / 1, one row per thread
-//               (= TMEM lane): tcgen05.ld of the S row, mask on boundary tiles,
-//               online softmax in base 2, P as bf16 pairs written back into the
-//               upper S columns of TMEM (tcgen05.st). The running max is only raised
-//               when a tile's max exceeds it by more than 2^8, so the O
-//               accumulator is rescaled in TMEM rarely; the final 1/l and LSE
-//               make the result exact either way. The row's scores are read
-//               from TMEM once and kept in registers.
-//   warp 8      TMA producer: both Q tiles once, then K and V tiles of 128 keys
-//               into a 2-stage ring (128-byte swizzle). The 4-D tensor maps are
-//               (d, head-or-stream*head, row, batch), so an INTRA stream is read
-//               as a contiguous causal problem (row stride n*H*D), with no copy.
-//   warp 9      allocates TMEM (2 x [S/P 128 columns | O D columns]) and walks
-//               the MMA loop as a whole warp (warp-uniform operands), one
-//               elected lane issuing every tcgen05.mma, in the order
-//                   PV_0(j), S_0(j+1), PV_1(j), S_1(j+1)
-//               so one tile's MMAs run while the other tile's softmax works.
+// One CTA = one 128-row query tile of one (batch, head, stream group); two CTAs
+// share an SM (256 TMEM columns and under 100 KB of shared memory each), so one
+// CTA's tensor-core work runs while the other's softmax, start-up or output
+// store does, and the two chains never wait on each other.
+//   warps 0-3   softmax, one row per thread (= TMEM lane): tcgen05.ld of the S
+//               row, mask on boundary tiles, online softmax in base 2, P as
+//               bf16 pairs written back into the upper S columns of TMEM
+//               (tcgen05.st). The running max is only raised when a tile's
+//               max exceeds it by more than 2^8, so the O accumulator is
+//               rescaled in TMEM rarely; the final 1/l and LSE make the result
+//               exact either way. The row's scores are read from TMEM once and
+//               kept in registers. Then the output: O/l as bf16 through the Q
+//               tile's shared memory to a TMA store, and the LSE.
+//   warp 4      TMA producer: the Q tile once, then K and V tiles of 128 keys
+//               (128-byte swizzle), one buffer each: K(j+1) streams in while
+//               S(j) is exponentiated, V(j+1) once PV(j) has read V(j). The 4-D
+//               tensor maps are (d, head-or-stream*head, row, batch), so an
+//               INTRA stream is read as a contiguous causal problem (row stride
+//               n*H*D), with no copy.
+//   warp 5      allocates TMEM ([S/P 128 columns | O D columns]) and walks the
+//               MMA loop as a whole warp (warp-uniform operands), one elected
+//               lane issuing every tcgen05.mma:
 //               S = Q K^T (M=128, N=128, both operands from shared memory);
 //               O += P V (M=128, N=D, P from TMEM, V MN-major from its TMA tile),
 //               issued in two halves of 64 keys: the softmax signals P of keys
-//               64-127 before it exponentiates keys 0-63, so half
-//               of PV runs under the rest of the softmax.
-// MMAs from one thread execute in order, so when S_q(j) is complete, PV_q(j-1)
+//               64-127 before it exponentiates keys 0-63, so half of PV runs
+//               under the rest of the softmax. S(j+1) follows PV(j).
+// MMAs from one thread execute in order, so when S(j) is complete, PV(j-1)
 // (issued before it) has finished reading P and updating O: the softmax may
 // then rescale O and overwrite P without another wait.
 // Every mbarrier wait is bounded; on expiry the kernel records HD_ERR_TIMEOUT,
@@ -49,11 +50,11 @@ namespace hd {
 
 namespace {
 
-constexpr int kBM = 128;  // query rows per tile (2 tiles per CTA)
-constexpr int kBN = 128;  // keys per K/V tile
-constexpr int kThreads = 320;
+constexpr int kBM = 128;        // query rows per CTA
+constexpr int kBN = 128;        // keys per K/V tile
+constexpr int kThreads = 192;   // warps 0-3 softmax, 4 TMA producer, 5 MMA issuer
 constexpr int kSub = 128 * 128;  // bytes of one [128 rows][64 bf16] swizzled sub-tile
-constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemCols = 256;
 constexpr float kRescaleLog2 = 8.f;  // raise the running max only past 2^8
 
 template <int D>
@@ -61,30 +62,23 @@ struct TcSmem {
   static constexpr int NSUB = D / 64;
   static constexpr int Q_BYTES = kBM * D * 2;
   static constexpr int KV_BYTES = kBN * D * 2;
-  static constexpr int Q_OFF = 0;                          // 2 query tiles
-  static constexpr int K_OFF = Q_OFF + 2 * Q_BYTES;        // 2 stages
-  static constexpr int V_OFF = K_OFF + 2 * KV_BYTES;       // 2 stages
-  static constexpr int BAR_OFF = V_OFF + 2 * KV_BYTES;
-  // q_full, k_full[2], v_full[2], kv_empty[2], s_full[2], p_hi[2], p_lo[2], o_final[2]
-  static constexpr int NBAR = 15;
+  static constexpr int Q_OFF = 0;
+  static constexpr int K_OFF = Q_OFF + Q_BYTES;
+  static constexpr int V_OFF = K_OFF + KV_BYTES;
+  static constexpr int BAR_OFF = V_OFF + KV_BYTES;
+  // q_full, k_full, v_full, k_empty, v_empty, s_full, p_hi, p_lo, o_final
+  static constexpr int NBAR = 9;
   static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;
   static constexpr int ABORT_OFF = SLOT_OFF + 4;
   static constexpr int USED = ABORT_OFF + 4 + 1024;
-  // at least 120 KB so that one CTA (one 512-column TMEM allocation) is resident per SM
-  static constexpr int TOTAL = USED > 120 * 1024 ? USED : 120 * 1024;
+  // at least 80 KB, so that at most two CTAs (2 x 256 TMEM columns) share an SM
+  static constexpr int TOTAL = USED > 80 * 1024 ? USED : 80 * 1024;
 };
 
 // p_hi: P of keys 64-127 written; p_lo: P of keys 0-63 written
-enum { B_QF = 0, B_KF = 1, B_VF = 3, B_KE = 5, B_SF = 7, B_PA = 9, B_PB = 11, B_OF = 13 };
+enum { B_QF = 0, B_KF = 1, B_VF = 2, B_KE = 3, B_VE = 4, B_SF = 5, B_PA = 6, B_PB = 7, B_OF = 8 };
 
-// A CTA takes the same query rows of two heads of one GQA group when the group
-// size is even (their K/V steps are identical), else two consecutive row tiles
-// of one head (the second one needs one K/V tile more on the causal diagonal).
-__host__ __device__ __forceinline__ bool fwd_head_pairs(const AttnParams& p) {
-  return (p.Hq / p.Hkv) % 2 == 0;
-}
-
-// Grid order of head-paired CTAs. Query-tile-major (the heaviest tiles of
+// Grid order. Query-tile-major (the heaviest tiles of
 // every problem first) balances short problems. For long full-causal ones
 // (no window, one stream group, at least 128 query tiles) it spreads the
 // CTAs running at once over every KV head, so each head's K/V tiles are read
@@ -97,7 +91,7 @@ __host__ __device__ __forceinline__ bool fwd_kv_major(const AttnParams& p, int n
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     attn_fwd_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                        const __grid_constant__ CUtensorMap tmO) {
@@ -111,84 +105,45 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + SM::ABORT_OFF);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // A timeout recorded by an earlier CTA (or call) is sticky until the status
-  // word is cleared: skip the work instead of waiting again.
   if (p.status && *reinterpret_cast<volatile int*>(p.status) == HD_ERR_TIMEOUT) return;
 
-  // ---- problem of this CTA: its two query tiles
   const int num_qt = (p.Lq + kBM - 1) / kBM;
-  const bool head_pair = fwd_head_pairs(p);
-  int b, grp, h0, h1, r00, r01;  // batch, stream group; head and first row of tile 0 / 1
-  if (head_pair && fwd_kv_major(p, num_qt)) {
-    // long full-causal problems: every CTA of one (batch, KV head) before the
-    // next one's, heaviest query tiles first inside it, so the CTAs running at
-    // once read the same KV head's tiles and keep them in L2
-    const int pairs = p.Hq / p.Hkv / 2;  // head pairs per KV head
-    const int per_kv = num_qt * pairs;
+  const int g = p.Hq / p.Hkv;
+  int b, grp, h, qt;
+  if (fwd_kv_major(p, num_qt)) {
+    const int per_kv = num_qt * g;
     const int bk = static_cast<int>(blockIdx.x / per_kv);
     const int rem = static_cast<int>(blockIdx.x % per_kv);
-    const int qt = num_qt - 1 - rem / pairs;
+    qt = num_qt - 1 - rem / g;
     grp = 0;
     b = bk / p.Hkv;
-    h0 = 2 * ((bk % p.Hkv) * pairs + rem % pairs);
-    h1 = h0 + 1;
-    r00 = r01 = qt * kBM;
-  } else if (head_pair) {
-    // the same 128 rows of two query heads that share a KV head: both tiles
-    // visit exactly the same K/V tiles
-    const int bhg = p.B * (p.Hq / 2) * p.groups;
-    const int qt = num_qt - 1 - static_cast<int>(blockIdx.x / bhg);  // heavy tiles first
-    int y = static_cast<int>(blockIdx.x % bhg);
-    grp = y % p.groups;
-    y /= p.groups;
-    h0 = 2 * (y % (p.Hq / 2));
-    h1 = h0 + 1;
-    b = y / (p.Hq / 2);
-    r00 = r01 = qt * kBM;
+    h = (bk % p.Hkv) * g + rem % g;
   } else {
-    // query tiles 2*pq and 2*pq+1 of one head
     const int bhg = p.B * p.Hq * p.groups;
-    const int num_pairs = (num_qt + 1) / 2;
-    const int pq = num_pairs - 1 - static_cast<int>(blockIdx.x / bhg);  // heavy pairs first
+    qt = num_qt - 1 - static_cast<int>(blockIdx.x / bhg);  // heavy tiles first
     int y = static_cast<int>(blockIdx.x % bhg);
     grp = y % p.groups;
     y /= p.groups;
-    h0 = h1 = y % p.Hq;
+    h = y % p.Hq;
     b = y / p.Hq;
-    r00 = 2 * pq * kBM;
-    r01 = r00 + kBM;
   }
-  const int hk = h0 / (p.Hq / p.Hkv);
+  const int r0 = qt * kBM;  // first query row of the tile
+  const int hk = h / g;
   const bool intra = p.mode == HD_INTRA;
-  const int jq0 = (intra && !p.final_only) ? grp * p.Hq + h0 : h0;
-  const int jq1 = (intra && !p.final_only) ? grp * p.Hq + h1 : h1;
+  const int jq = (intra && !p.final_only) ? grp * p.Hq + h : h;
   const int jk = intra ? (p.final_only ? p.n - 1 : grp) * p.Hkv + hk : hk;
-  // K/V tile range [lo_q, hi_q] of each query tile (empty when the tile has no rows)
-  int lo[2], hi[2];
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    const int rq = q ? r01 : r00;
-    if (rq >= p.Lq) {
-      lo[q] = 1;
-      hi[q] = 0;
-      continue;
-    }
-    const int rl = min(rq + kBM, p.Lq) - 1;
-    lo[q] = max(0, p.a * rq + p.bb - p.win + 1) / kBN;
-    hi[q] = min(p.Lk - 1, p.a * rl + p.bb) / kBN;
-  }
-  const int kt_lo = lo[1] <= hi[1] ? min(lo[0], lo[1]) : lo[0];
-  const int kt_hi = max(hi[0], hi[1]);
+  const int rq_last = min(r0 + kBM, p.Lq) - 1;
+  // key tiles [kt_lo, kt_hi] hold every key some row of the tile sees
+  const int kt_lo = max(0, p.a * r0 + p.bb - p.win + 1) / kBN;
+  const int kt_hi = min(p.Lk - 1, p.a * rq_last + p.bb) / kBN;
   const int nkv = kt_hi - kt_lo + 1;
-  auto in_range = [&](int q, int j) { return j >= lo[q] && j <= hi[q]; };
 
   if (tid == 0) {
-    // softmax warps arrive once per warp (4); everything else arrives once
-    for (int i = 0; i < SM::NBAR; ++i) tc::mbar_init(bar(i), (i >= B_PA && i < B_PB + 2) ? 4 : 1);
+    for (int i = 0; i < SM::NBAR; ++i) tc::mbar_init(bar(i), (i == B_PA || i == B_PB) ? 4 : 1);
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == 5) {
     tc::tmem_alloc(sbase + SM::SLOT_OFF, kTmemCols);
     tc::tmem_relinquish();
   }
@@ -196,123 +151,94 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sgen + SM::SLOT_OFF);
-  // tile q: S at 256q (P, as bf16 pairs, in its columns 64..127), O at 256q + 128
+  // S at column 0 (P, as bf16 pairs, in its columns 64..127), O at column 128
 
-  if (warp == 8) {
+  if (warp == 4) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tc::tma_prefetch_desc(&tmQ);
       tc::tma_prefetch_desc(&tmK);
       tc::tma_prefetch_desc(&tmV);
-      tc::mbar_expect_tx(bar(B_QF), 2 * SM::Q_BYTES);
+      tc::mbar_expect_tx(bar(B_QF), SM::Q_BYTES);
 #pragma unroll
-      for (int q = 0; q < 2; ++q)
-#pragma unroll
-        for (int s = 0; s < NSUB; ++s)
-          tc::tma_load_4d(sQ + q * SM::Q_BYTES + s * kSub, &tmQ, bar(B_QF), s * 64, q ? jq1 : jq0,
-                          q ? r01 : r00, b);
+      for (int s = 0; s < NSUB; ++s) tc::tma_load_4d(sQ + s * kSub, &tmQ, bar(B_QF), s * 64, jq, r0, b);
       for (int i = 0; i < nkv; ++i) {
-        const int st = i & 1;
-        if (!tc::mbar_wait(bar(B_KE + st), ((i >> 1) & 1) ^ 1, abort_flag, p.status)) break;
         const int c0 = (kt_lo + i) * kBN;
-        tc::mbar_expect_tx(bar(B_KF + st), SM::KV_BYTES);
+        // K(i) once S(i-1) has read K(i-1); V(i) once PV(i-1) has read V(i-1)
+        if (i > 0 && !tc::mbar_wait(bar(B_KE), (i - 1) & 1, abort_flag, p.status)) break;
+        tc::mbar_expect_tx(bar(B_KF), SM::KV_BYTES);
 #pragma unroll
-        for (int s = 0; s < NSUB; ++s)
-          tc::tma_load_4d(sK + st * SM::KV_BYTES + s * kSub, &tmK, bar(B_KF + st), s * 64, jk, c0, b);
-        tc::mbar_expect_tx(bar(B_VF + st), SM::KV_BYTES);
+        for (int s = 0; s < NSUB; ++s) tc::tma_load_4d(sK + s * kSub, &tmK, bar(B_KF), s * 64, jk, c0, b);
+        if (i > 0 && !tc::mbar_wait(bar(B_VE), (i - 1) & 1, abort_flag, p.status)) break;
+        tc::mbar_expect_tx(bar(B_VF), SM::KV_BYTES);
 #pragma unroll
-        for (int s = 0; s < NSUB; ++s)
-          tc::tma_load_4d(sV + st * SM::KV_BYTES + s * kSub, &tmV, bar(B_VF + st), s * 64, jk, c0, b);
+        for (int s = 0; s < NSUB; ++s) tc::tma_load_4d(sV + s * kSub, &tmV, bar(B_VF), s * 64, jk, c0, b);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 5) {
     // ------------------------------------------------------------- MMA issuer
-    {  // the whole warp walks the issue loop; one elected lane issues
-      constexpr uint32_t idS = tc::idesc_bf16_f32(kBM, kBN, 0, 0);
-      constexpr uint32_t idO = tc::idesc_bf16_f32(kBM, D, 0, 1);
-      auto issue_S = [&](int q, int st) {
+    constexpr uint32_t idS = tc::idesc_bf16_f32(kBM, kBN, 0, 0);
+    constexpr uint32_t idO = tc::idesc_bf16_f32(kBM, D, 0, 1);
+    auto issue_S = [&]() {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
-          tc::mma_ss_elect(tmem + 256 * q, tc::smem_desc_sw128(sQ + q * SM::Q_BYTES + off, 16, 1024),
-                           tc::smem_desc_sw128(sK + st * SM::KV_BYTES + off, 16, 1024), idS, kk > 0);
-        }
-        tc::mma_commit_elect(bar(B_SF + q));
-      };
-      int pf_count[2] = {0, 0};
-      bool ok = tc::mbar_wait_warp(bar(B_QF), 0, abort_flag, p.status) &&
-                tc::mbar_wait_warp(bar(B_KF), 0, abort_flag, p.status);
-      if (ok) {
-        tc::tc_fence_after();
-#pragma unroll
-        for (int q = 0; q < 2; ++q)
-          if (in_range(q, kt_lo)) issue_S(q, 0);
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
+        tc::mma_ss_elect(tmem, tc::smem_desc_sw128(sQ + off, 16, 1024), tc::smem_desc_sw128(sK + off, 16, 1024),
+                         idS, kk > 0);
       }
-      for (int i = 0; ok && i < nkv; ++i) {
-        const int j = kt_lo + i, st = i & 1, s1 = (i + 1) & 1;
-        bool v_ready = false, k_next_ready = false;
+      tc::mma_commit_elect(bar(B_SF));
+      tc::mma_commit_elect(bar(B_KE));
+    };
+    bool ok = nkv > 0 && tc::mbar_wait_warp(bar(B_QF), 0, abort_flag, p.status) &&
+              tc::mbar_wait_warp(bar(B_KF), 0, abort_flag, p.status);
+    if (ok) {
+      tc::tc_fence_after();
+      issue_S();
+    }
+    for (int i = 0; ok && i < nkv; ++i) {
+      const int j = kt_lo + i;
+      ok = tc::mbar_wait_warp(bar(B_PA), i & 1, abort_flag, p.status) &&
+           tc::mbar_wait_warp(bar(B_VF), i & 1, abort_flag, p.status);
+      if (!ok) break;
+      tc::tc_fence_after();
 #pragma unroll
-        for (int q = 0; q < 2 && ok; ++q) {
-          if (in_range(q, j)) {
-            // PV in two halves of 64 keys: keys 64-127 as soon as their P is
-            // written, while the softmax still works on keys 0-63
-            ok = tc::mbar_wait_warp(bar(B_PA + q), pf_count[q] & 1, abort_flag, p.status);
-            if (ok && !v_ready) ok = tc::mbar_wait_warp(bar(B_VF + st), (i >> 1) & 1, abort_flag, p.status);
-            if (!ok) break;
-            v_ready = true;
-            tc::tc_fence_after();
+      for (int kk = kBN / 32; kk < kBN / 16; ++kk)
+        tc::mma_ts_elect(tmem + 128, tmem + 64 + kk * 8, tc::smem_desc_sw128(sV + kk * 2048, kSub, 1024), idO,
+                         (j > kt_lo || kk > kBN / 32) ? 1u : 0u);
+      ok = tc::mbar_wait_warp(bar(B_PB), i & 1, abort_flag, p.status);
+      if (!ok) break;
+      tc::tc_fence_after();
 #pragma unroll
-            for (int kk = kBN / 32; kk < kBN / 16; ++kk)
-              tc::mma_ts_elect(tmem + 256 * q + 128, tmem + 256 * q + 64 + kk * 8,
-                               tc::smem_desc_sw128(sV + st * SM::KV_BYTES + kk * 2048, kSub, 1024), idO,
-                               (j > lo[q] || kk > kBN / 32) ? 1u : 0u);
-            ok = tc::mbar_wait_warp(bar(B_PB + q), pf_count[q] & 1, abort_flag, p.status);
-            if (!ok) break;
-            ++pf_count[q];
-            tc::tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < kBN / 32; ++kk)
-              tc::mma_ts_elect(tmem + 256 * q + 128, tmem + 256 * q + 64 + kk * 8,
-                               tc::smem_desc_sw128(sV + st * SM::KV_BYTES + kk * 2048, kSub, 1024), idO, 1u);
-            if (j == hi[q]) tc::mma_commit_elect(bar(B_OF + q));
-          }
-          if (in_range(q, j + 1)) {
-            if (!k_next_ready) {
-              ok = tc::mbar_wait_warp(bar(B_KF + s1), ((i + 1) >> 1) & 1, abort_flag, p.status);
-              if (!ok) break;
-              k_next_ready = true;
-              tc::tc_fence_after();
-            }
-            issue_S(q, s1);
-          }
-        }
-        tc::mma_commit_elect(bar(B_KE + st));
+      for (int kk = 0; kk < kBN / 32; ++kk)
+        tc::mma_ts_elect(tmem + 128, tmem + 64 + kk * 8, tc::smem_desc_sw128(sV + kk * 2048, kSub, 1024), idO,
+                         1u);
+      tc::mma_commit_elect(bar(B_VE));
+      if (j == kt_hi) tc::mma_commit_elect(bar(B_OF));
+      if (i + 1 < nkv) {
+        ok = tc::mbar_wait_warp(bar(B_KF), (i + 1) & 1, abort_flag, p.status);
+        if (!ok) break;
+        tc::tc_fence_after();
+        issue_S();
       }
     }
   } else {
-    // ------------------------------------------------------ softmax warpgroups
-    const int q = warp >> 2;  // query tile of this warpgroup
-    const int row = tid & 127;
-    const int rq0 = q ? r01 : r00;  // first row of this warpgroup's tile
-    const int hq = q ? h1 : h0, jq = q ? jq1 : jq0;
-    const int r = rq0 + row;
-    const uint32_t tq = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + 256 * q + tq, tO = tS + 128;
-    const int rq_last = min(rq0 + kBM, p.Lq) - 1;
+    const int row = tid;
+    const int r = r0 + row;
+    const uint32_t tq = static_cast<uint32_t>(warp * 32) << 16;  // this warp's TMEM lanes
+    const uint32_t tS = tmem + tq, tO = tS + 128;
     const int hi_r = p.a * r + p.bb;
     const int lo_r = hi_r - p.win;
-    const int my_lo = q ? lo[1] : lo[0], my_hi = q ? hi[1] : hi[0];
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     int t = 0;
-    for (int j = my_lo; j <= my_hi; ++j, ++t) {
-      if (!tc::mbar_wait(bar(B_SF + q), t & 1, abort_flag, p.status)) { ok = false; break; }
+    for (int j = kt_lo; j <= kt_hi; ++j, ++t) {
+      if (!tc::mbar_wait(bar(B_SF), t & 1, abort_flag, p.status)) { ok = false; break; }
       tc::tc_fence_after();
       const int c0 = j * kBN;
-      const bool full = (c0 + kBN - 1 <= p.a * rq0 + p.bb) &&
+      const bool full = (c0 + kBN - 1 <= p.a * r0 + p.bb) &&
                         (c0 > p.a * rq_last + p.bb - p.win) && (c0 + kBN <= p.Lk);
       // The row's 128 scores are read from TMEM once and stay in registers
-      // (167 registers per thread, under the 168 that 10 warps allow).
+      // (159 registers per thread, under the 170 that two CTAs of 6 warps allow).
       // P goes to columns 64..127 as bf16 pairs (keys 0-63 -> 64..95,
       // keys 64-127 -> 96..127), i.e. only over scores already read.
       auto mask32 = [&](uint32_t* v, int k0) {
@@ -394,21 +320,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tmem_wait_st();
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(bar(B_PA + q));
+      if (lane == 0) tc::mbar_arrive(bar(B_PA));
       exp32(v, 64, m_use);
       exp32(v + 32, 80, m_use);
       tc::tmem_wait_st();
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(bar(B_PB + q));
+      if (lane == 0) tc::mbar_arrive(bar(B_PB));
     }
-    const bool has_rows = my_lo <= my_hi;
-    if (ok && has_rows && !*abort_flag) ok = tc::mbar_wait(bar(B_OF + q), 0, abort_flag, p.status);
-    const uint32_t sQq = sQ + q * SM::Q_BYTES;
+    const bool has_rows = nkv > 0;
+    if (ok && has_rows && !*abort_flag) ok = tc::mbar_wait(bar(B_OF), 0, abort_flag, p.status);
     if (ok && has_rows) {
       tc::tc_fence_after();
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      // O row -> bf16 -> shared memory (this tile's Q space, same swizzled layout)
+      // O row -> bf16 -> shared memory (the Q tile's space, same swizzled layout)
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -418,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < 4; ++k) {
           const int d8 = c * 4 + k;  // chunk of 8 columns
           const float* f = reinterpret_cast<const float*>(o + k * 8);
-          const uint32_t addr = sQq + (d8 >> 3) * kSub + row * 128 + (((d8 & 7) ^ (row & 7)) << 4);
+          const uint32_t addr = sQ + (d8 >> 3) * kSub + row * 128 + (((d8 & 7) ^ (row & 7)) << 4);
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr),
                        "r"(pack_bf16(f[0] * inv, f[1] * inv)), "r"(pack_bf16(f[2] * inv, f[3] * inv)),
                        "r"(pack_bf16(f[4] * inv, f[5] * inv)), "r"(pack_bf16(f[6] * inv, f[7] * inv))
@@ -426,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (r < p.Lq) {
-        const long long li = (static_cast<long long>(b) * p.Hq + hq) * p.Sq +
+        const long long li = (static_cast<long long>(b) * p.Hq + h) * p.Sq +
                              static_cast<long long>(grp) * p.qs_step +
                              static_cast<long long>(r) * p.q_rstride;
         if (in_bounds(li, 1, p.ext_lse, p.status))
@@ -434,17 +359,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc::fence_async_smem();
     }
-    if (q == 0) asm volatile("bar.sync 1, 128;\n" ::: "memory");
-    else asm volatile("bar.sync 2, 128;\n" ::: "memory");
+    asm volatile("bar.sync 1, 128;\n" ::: "memory");  // the softmax warps only
     if (row == 0 && ok && has_rows && !*abort_flag) {
 #pragma unroll
-      for (int s = 0; s < NSUB; ++s) tc::tma_store_4d(&tmO, sQq + s * kSub, s * 64, jq, rq0, b);
+      for (int s = 0; s < NSUB; ++s) tc::tma_store_4d(&tmO, sQ + s * kSub, s * 64, jq, r0, b);
       tc::tma_store_commit_and_wait();
     }
   }
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 5) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, kTmemCols);
   }
@@ -512,8 +436,7 @@ cudaError_t launch_tc_d(const AttnParams& p, cudaStream_t stream) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const long long num_qt = (p.Lq + kBM - 1) / kBM;
-  const long long blocks = fwd_head_pairs(p) ? num_qt * p.B * (p.Hq / 2) * p.groups
-                                             : (num_qt + 1) / 2 * p.B * p.Hq * p.groups;
+  const long long blocks = num_qt * p.B * p.Hq * p.groups;
   attn_fwd_tc_kernel<D><<<static_cast<unsigned>(blocks), kThreads, smem, stream>>>(p, mq, mk, mv, mo);
   return cudaGetLastError();
 }

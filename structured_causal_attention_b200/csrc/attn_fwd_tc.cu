@@ -78,14 +78,15 @@ struct TcSmem {
 // p_hi: P of keys 64-127 written; p_lo: P of keys 0-63 written
 enum { B_QF = 0, B_KF = 1, B_VF = 2, B_KE = 3, B_VE = 4, B_SF = 5, B_PA = 6, B_PB = 7, B_OF = 8 };
 
-// Grid order. Query-tile-major (the heaviest tiles of
-// every problem first) balances short problems. For long full-causal ones
-// (no window, one stream group, at least 128 query tiles) it spreads the
-// CTAs running at once over every KV head, so each head's K/V tiles are read
-// by CTAs far apart in time and come back from DRAM: 203 GB of DRAM reads
-// for one forward at 131072 positions, whose algorithmic bytes are 2.7 GB.
-// Those problems take a KV-head-major order instead: 3.2 GB of reads, an L2
-// hit rate of 99 % against 39 %, and 6 % less time at the power cap.
+// Grid order, heaviest query tiles first. Query-tile-major order balances
+// short problems. For long full-causal ones (no window, one stream group, at
+// least 128 query tiles) it spreads the CTAs running at once over every KV
+// head, so each head's K/V tiles are read by CTAs far apart in time and come
+// back from DRAM (about 200 GB of reads for one forward at 131072 positions,
+// whose algorithmic bytes are 2.7 GB). Those problems take a KV-head-major
+// order instead, and inside one KV head the heads of its group at each query
+// tile: 3.2 GB of reads at an L2 hit rate of 99 %, and 4 % less time at the
+// power cap.
 __host__ __device__ __forceinline__ bool fwd_kv_major(const AttnParams& p, int num_qt) {
   return p.win >= p.Lk && p.groups == 1 && num_qt >= 128;
 }
@@ -238,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const bool full = (c0 + kBN - 1 <= p.a * r0 + p.bb) &&
                         (c0 > p.a * rq_last + p.bb - p.win) && (c0 + kBN <= p.Lk);
       // The row's 128 scores are read from TMEM once and stay in registers
-      // (159 registers per thread, under the 170 that two CTAs of 6 warps allow).
+      // (158 registers per thread, under the 168 that two CTAs of 6 warps allow).
       // P goes to columns 64..127 as bf16 pairs (keys 0-63 -> 64..95,
       // keys 64-127 -> 96..127), i.e. only over scores already read.
       auto mask32 = [&](uint32_t* v, int k0) {

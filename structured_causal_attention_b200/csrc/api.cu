@@ -248,7 +248,7 @@ int hd_expand_embed(const int32_t* ids, const void* tables, void* out, int B, in
   if (elem_bytes == 1 && row_bytes % 2 != 0) return HD_ERR_UNSUPPORTED;
   if ((reinterpret_cast<uintptr_t>(tables) | reinterpret_cast<uintptr_t>(out)) % 2 != 0)
     return HD_ERR_INVALID_ARG;
-  return from_cuda(launch_expand(ids, tables, out, B, L, n, V, row_bytes, status_ptr(),
+  return from_cuda(launch_expand(ids, tables, out, B, L, n, V, row_bytes, sm_count(), status_ptr(),
                                  static_cast<cudaStream_t>(stream)));
 }
 
@@ -276,7 +276,7 @@ int hd_rope_expanded(void* q, void* k, const int32_t* token_offset, int B, int L
   p.D = D;
   p.final_only = final_stream_queries_only;
   p.log2_base = std::log2(base);
-  return from_cuda(launch_rope(p, static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_rope(p, sm_count(), static_cast<cudaStream_t>(stream)));
 }
 
 int hd_final_readout(const void* x, void* out, int B, int L, int n, int d, int elem_bytes,
@@ -288,7 +288,7 @@ int hd_final_readout(const void* x, void* out, int B, int L, int n, int d, int e
   if (!aligned16(x) || !aligned16(out)) return HD_ERR_INVALID_ARG;
   const long long row_bytes = static_cast<long long>(d) * elem_bytes;
   if (row_bytes % 16 != 0) return HD_ERR_UNSUPPORTED;
-  return from_cuda(launch_final_readout(x, out, static_cast<long long>(B) * L, n, row_bytes,
+  return from_cuda(launch_final_readout(x, out, static_cast<long long>(B) * L, n, row_bytes, sm_count(),
                                         status_ptr(), static_cast<cudaStream_t>(stream)));
 }
 

@@ -59,10 +59,10 @@ __global__ void __launch_bounds__(256) expand_kernel(const int32_t* __restrict__
 
 template <typename Vec, int UNROLL>
 cudaError_t launch_vec(const int32_t* ids, const void* tables, void* out, int B, int L, int n,
-                       int V, long long row_bytes, int* status, cudaStream_t stream) {
+                       int V, long long row_bytes, int sms, int* status, cudaStream_t stream) {
   const long long nrows = static_cast<long long>(B) * L * n;
   long long blocks = (nrows + 7) / 8;
-  const long long cap = 148LL * 8 * 16;  // grid-stride beyond 16 waves of 8 warps
+  const long long cap = static_cast<long long>(sms) * 8 * 16;  // grid-stride beyond 16 waves of 8 warps
   if (blocks > cap) blocks = cap;
   expand_kernel<Vec, UNROLL><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
       ids, static_cast<const uint8_t*>(tables), static_cast<uint8_t*>(out), B, L, n, V, row_bytes,
@@ -73,14 +73,14 @@ cudaError_t launch_vec(const int32_t* ids, const void* tables, void* out, int B,
 }  // namespace
 
 cudaError_t launch_expand(const int32_t* ids, const void* tables, void* out, int B, int L, int n,
-                          int V, long long row_bytes, int* status, cudaStream_t stream) {
+                          int V, long long row_bytes, int sms, int* status, cudaStream_t stream) {
   const bool a16 = (reinterpret_cast<uintptr_t>(tables) % 16 == 0) &&
                    (reinterpret_cast<uintptr_t>(out) % 16 == 0) && (row_bytes % 16 == 0);
-  if (a16) return launch_vec<uint4, 4>(ids, tables, out, B, L, n, V, row_bytes, status, stream);
+  if (a16) return launch_vec<uint4, 4>(ids, tables, out, B, L, n, V, row_bytes, sms, status, stream);
   const bool a4 = (reinterpret_cast<uintptr_t>(tables) % 4 == 0) &&
                   (reinterpret_cast<uintptr_t>(out) % 4 == 0) && (row_bytes % 4 == 0);
-  if (a4) return launch_vec<uint32_t, 4>(ids, tables, out, B, L, n, V, row_bytes, status, stream);
-  return launch_vec<uint16_t, 4>(ids, tables, out, B, L, n, V, row_bytes, status, stream);
+  if (a4) return launch_vec<uint32_t, 4>(ids, tables, out, B, L, n, V, row_bytes, sms, status, stream);
+  return launch_vec<uint16_t, 4>(ids, tables, out, B, L, n, V, row_bytes, sms, status, stream);
 }
 
 }  // namespace hd

@@ -56,7 +56,7 @@ struct RopeParams {
   int B, S, Sq, n, Hq, Hkv, D, final_only;
   double log2_base;
 };
-cudaError_t launch_rope(const RopeParams& p, cudaStream_t stream);
+cudaError_t launch_rope(const RopeParams& p, int sms, cudaStream_t stream);
 
 struct LmHeadParams {
   const int32_t* labels;  // [R]
@@ -81,11 +81,11 @@ cudaError_t launch_lm_head_ce_bwd(LmHeadParams p, const void* x, const void* w, 
 cudaError_t launch_lm_head_ce(LmHeadParams p, const void* x, const void* w, int n, int num_sms,
                               cudaStream_t stream);
 cudaError_t launch_final_readout(const void* x, void* out, long long rows, int n,
-                                 long long row_bytes, int* status, cudaStream_t stream);
+                                 long long row_bytes, int sms, int* status, cudaStream_t stream);
 
 cudaError_t launch_wait_timeout(long long limit_cycles, int* status, cudaStream_t stream);
 
 cudaError_t launch_expand(const int32_t* ids, const void* tables, void* out, int B, int L, int n,
-                          int V, long long row_bytes, int* status, cudaStream_t stream);
+                          int V, long long row_bytes, int sms, int* status, cudaStream_t stream);
 
 }  // namespace hd

@@ -615,9 +615,10 @@ cudaError_t launch_lm_head_ce_bwd(LmHeadParams p, const void* x, const void* w, 
 }
 
 cudaError_t launch_final_readout(const void* x, void* out, long long rows, int n,
-                                 long long row_bytes, int* status, cudaStream_t stream) {
+                                 long long row_bytes, int sms, int* status, cudaStream_t stream) {
   long long blocks = (rows + 7) / 8;
-  if (blocks > 148LL * 16) blocks = 148LL * 16;
+  const long long cap = static_cast<long long>(sms) * 16;  // grid-stride beyond 16 blocks per SM
+  if (blocks > cap) blocks = cap;
   final_readout_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
       static_cast<const uint8_t*>(x), static_cast<uint8_t*>(out), rows, n, row_bytes, status);
   return cudaGetLastError();

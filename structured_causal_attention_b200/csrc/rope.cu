@@ -117,12 +117,12 @@ __global__ void __launch_bounds__(kRopeThreads) rope_kernel(RopeParams p) {
 
 }  // namespace
 
-cudaError_t launch_rope(const RopeParams& p, cudaStream_t stream) {
+cudaError_t launch_rope(const RopeParams& p, int sms, cudaStream_t stream) {
   const int J = p.D / 16;
   const long long tasks = (p.q ? static_cast<long long>(p.B) * p.Sq * J : 0) +
                           (p.k ? static_cast<long long>(p.B) * p.S * J : 0);
   long long blocks = (tasks + kRopeThreads - 1) / kRopeThreads;
-  const long long cap = 148LL * 8;  // 8 resident 256-thread blocks per SM, grid-stride beyond
+  const long long cap = static_cast<long long>(sms) * 8;  // 8 resident 256-thread blocks per SM, grid-stride beyond
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   static_assert(kRopeThreads % 16 == 0, "the grid stride must be a multiple of D/16 <= 16");

@@ -57,7 +57,8 @@ def test_default_step_runs_every_configuration_at_its_sizes():
     assert (sizes["c4"]["B"], sizes["c4"]["n"] * sizes["c4"]["L"]) == (1, 131072)
     assert (sizes["c5b8"]["B"], sizes["c5b64"]["B"], sizes["c5b8"]["T"]) == (8, 64, 16384)
     op = {o["name"]: o for _, _, ops in parts for o in ops}
-    # 4a: 131072 (131072 + 1) / 2 pairs per head, 32 heads, 4 * D FLOPs each (BASELINE: 140.7 TFLOP)
+    # 4a: 131072 (131072 + 1) / 2 pairs per head, 32 heads, 4 * D FLOPs each (140.7 TFLOP, the
+    # published count for this configuration)
     assert op["c4.fwd_cross_full"]["flops"] == 4 * 128 * 32 * 131072 * 131073 // 2
     assert abs(op["c4.fwd_cross_full"]["flops"] / 1e12 - 140.7) < 0.1
     # decode B8: K and V of 65540 cache rows, 8 heads, D128, bf16 (2.148 GB)

@@ -364,11 +364,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // ---- warpgroup 0: dK (scaled), warpgroup 1: dV; TMEM -> bf16 -> shared
     // memory (the Q / dO stages) -> TMA store
-    if (ok && !*abort_flag && total > 0) ok = tc::mbar_wait(bar(B_END), 0, abort_flag, p.status);
+    // warp-uniform (the tcgen05.ld below needs the whole warp)
+    if (total > 0) ok = tc::mbar_wait_warp(bar(B_END), 0, abort_flag, p.status) && ok;
+    ok = __all_sync(0xffffffffu, ok && !*abort_flag);
     const uint32_t src = sw == 0 ? tdK : tdV;
     const uint32_t dst = sw == 0 ? sQ : sDO;  // kQS x NSUB x [64][64] >= NSUB x [128][64]
     const float sc = sw == 0 ? p.scale : 1.f;
-    if (ok && !*abort_flag) {
+    if (ok) {
       tc::tc_fence_after();
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {

@@ -330,7 +330,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (lane == 0) tc::mbar_arrive(bar(B_PB));
     }
     const bool has_rows = nkv > 0;
-    if (ok && has_rows && !*abort_flag) ok = tc::mbar_wait(bar(B_OF), 0, abort_flag, p.status);
+    // warp-uniform, every lane taking part (the tcgen05.ld of O below needs
+    // the whole warp)
+    if (has_rows) ok = tc::mbar_wait_warp(bar(B_OF), 0, abort_flag, p.status) && ok;
+    ok = __all_sync(0xffffffffu, ok);
     if (ok && has_rows) {
       tc::tc_fence_after();
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;

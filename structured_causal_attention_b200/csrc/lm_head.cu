@@ -187,7 +187,7 @@ __global__ void __launch_bounds__(kLThreads, 1)
 #pragma unroll
         for (int h = 0; h < 2; ++h) lse2[h] = row[h] < p.R ? __ldg(p.lse_in + row[h]) * kLog2e : 0.f;
       }
-      if (!tc::mbar_wait(bar(LB_ACC_FULL), ui & 1, abort_flag, p.status)) break;
+      if (!tc::mbar_wait_warp(bar(LB_ACC_FULL), ui & 1, abort_flag, p.status)) break;
       tc::tc_fence_after();
       if constexpr (kGrad) {
 #pragma unroll
@@ -390,7 +390,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
       const int buf = ui & 1;
       const int m0 = static_cast<int>(u / p.ntn) * kGM, n0 = static_cast<int>(u % p.ntn) * kGN;
       const int r = m0 + quarter * 32 + lane;
-      if (!tc::mbar_wait(bar(GB_AF + buf), (ui >> 1) & 1, abort_flag, p.status)) break;
+      if (!tc::mbar_wait_warp(bar(GB_AF + buf), (ui >> 1) & 1, abort_flag, p.status)) break;
       tc::tc_fence_after();
       for (int c = 0; c < kGN / 32; ++c) {
         uint32_t x[32];
